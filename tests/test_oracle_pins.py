@@ -1,0 +1,382 @@
+"""Pins for the CPU oracle, against things other than the oracle itself.
+
+Each test ties one oracle function to something fixed outside it: hand-derived
+golden fixtures (``tests/golden/``), brute-force search, closed forms, exact
+rational arithmetic, or invariants the method guarantees. A plausible slip in
+the oracle (a swapped min/max, a floor for a rint, a transposed operand, a
+fold applied the wrong way round, a wrong index in the layout) fails one of
+them. None of these tests needs a GPU.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import awq_oracle as O
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _f16_bits(a):
+    return np.asarray(a, dtype=np.float16).view(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# quantizer: hand-derived groups
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("case", _load("quantizer_hand_cases.json")["groups"], ids=lambda c: c["name"])
+def test_quantizer_hand_cases(case):
+    vals = list(case["values"]) + [case["fill"]] * (128 - len(case["values"]))
+    W = np.array([vals], dtype=np.float16)
+    assert np.all(W.astype(np.float64) == np.array([vals])), "fixture values must be fp16-exact"
+    q, S, z = O.quantize_groups(W)
+    expect = list(case["codes"]) + [case["fill_code"]] * (128 - len(case["codes"]))
+    assert q[0].tolist() == expect
+    assert int(_f16_bits(S)[0, 0]) == int(case["scale_bits"], 16)
+    assert int(z[0, 0]) == case["zero"]
+
+
+def test_quantizer_groups_are_independent_and_rows_too():
+    """Two hand groups side by side in one row, and stacked rows, give the same results."""
+    cases = _load("quantizer_hand_cases.json")["groups"]
+    rows = []
+    for c in cases:
+        rows.append(list(c["values"]) + [c["fill"]] * (128 - len(c["values"])))
+    a = np.array(rows, dtype=np.float16)
+    wide = np.concatenate([a, a[::-1]], axis=1)            # [n, 256]: 2 groups per row
+    q, S, z = O.quantize_groups(wide)
+    q1, S1, z1 = O.quantize_groups(a)
+    q2, S2, z2 = O.quantize_groups(a[::-1])
+    assert np.array_equal(q[:, :128], q1) and np.array_equal(q[:, 128:], q2)
+    assert np.array_equal(_f16_bits(S[:, 0]), _f16_bits(S1[:, 0]))
+    assert np.array_equal(_f16_bits(S[:, 1]), _f16_bits(S2[:, 0]))
+    assert np.array_equal(z[:, 0], z1[:, 0]) and np.array_equal(z[:, 1], z2[:, 0])
+
+
+# ----------------------------------------------------------------------------
+# quantizer: brute-force nearest level
+# ----------------------------------------------------------------------------
+def _brute_codes(w32, S16):
+    """q = the level c in 0..15 whose value (c - z) is nearest to w/S (fp32 quotient).
+
+    z itself is the integer in 0..15 nearest to -lo/S. Ties go to the even
+    integer (of c - z, resp. of z), which is what round-half-even means.
+    """
+    Sf = np.float32(S16)
+    lo = np.float32(np.min(w32))
+    t = float(np.float32(-lo) / Sf)
+    best = None
+    for c in range(16):
+        d = abs(t - c)
+        key = (d, c % 2)
+        if best is None or key < best[0]:
+            best = (key, c)
+    zb = best[1]
+    out = []
+    for w in w32:
+        v = float(np.float32(w) / Sf)
+        best = None
+        for c in range(16):
+            d = abs(v - (c - zb))
+            key = (d, (c - zb) % 2)
+            if best is None or key < best[0]:
+                best = (key, c)
+        out.append(best[1])
+    return np.array(out, dtype=np.uint8), zb
+
+
+def test_quantizer_brute_force_random_groups():
+    rng = np.random.default_rng(1234)
+    for trial in range(60):
+        kind = trial % 4
+        if kind == 0:
+            w = rng.standard_normal(128) * 0.02
+        elif kind == 1:
+            w = rng.standard_normal(128) * 3.0 + rng.uniform(-2, 2)
+        elif kind == 2:
+            w = rng.uniform(0.5, 1.5, 128)           # all positive: z clamps at 0
+        else:
+            w = -rng.uniform(0.5, 1.5, 128)          # all negative: z clamps at 15
+        W = w.astype(np.float16)[None, :]
+        q, S, z = O.quantize_groups(W)
+        qb, zb = _brute_codes(W[0].astype(np.float32), S[0, 0])
+        assert int(z[0, 0]) == zb
+        assert np.array_equal(q[0], qb), f"trial {trial}"
+
+
+def test_quantizer_exhaustive_fp16_grid_unit_scale():
+    """Every finite fp16 value in [-7, 8] placed in a group whose min/max are -7 and 8.
+
+    Then S = 1, z = 7 and the code of w must be clamp(rint(w) + 7): brute
+    force over the 16 levels decides it, ties to the even level.
+    """
+    bits = np.arange(0x10000, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(np.float16)
+    vals = vals[np.isfinite(vals)]
+    vals = vals[(vals >= -7) & (vals <= 8)]
+    vals = np.unique(vals.astype(np.float32))        # one -0/0 only
+    n = len(vals)
+    per = 126
+    rows = -(-n // per)
+    W = np.zeros((rows, 128), dtype=np.float16)
+    W[:, 0] = -7
+    W[:, 1] = 8
+    flat = np.zeros(rows * per, dtype=np.float32)
+    flat[:n] = vals
+    W[:, 2:] = flat.reshape(rows, per).astype(np.float16)
+    q, S, z = O.quantize_groups(W)
+    assert np.all(S.astype(np.float32) == 1.0) and np.all(z == 7)
+    got = q[:, 2:].reshape(-1)[:n]
+    # brute force with S = 1, z = 7 (v = w exactly)
+    levels = np.arange(16, dtype=np.float64) - 7
+    d = np.abs(vals.astype(np.float64)[:, None] - levels[None, :])
+    dmin = d.min(axis=1, keepdims=True)
+    cand = (d == dmin)
+    even = (np.mod(levels, 2) == 0)[None, :]
+    pick = np.where(cand & even, 1, 0) * 2 + np.where(cand, 1, 0)
+    expect = np.argmax(pick, axis=1)
+    assert np.array_equal(got.astype(np.int64), expect)
+
+
+# ----------------------------------------------------------------------------
+# quantizer: invariants on the synthetic recipe
+# ----------------------------------------------------------------------------
+def test_quantizer_invariants_on_recipe():
+    x, W = workloads.random_case(7, 4, 256, 1024)
+    s = O.activation_scale(x)
+    wf = O.fold_weights(W, s)
+    q, S, z = O.quantize_groups(wf)
+    assert q.dtype == np.uint8 and q.max() <= 15 and z.max() <= 15
+    N, K = wf.shape
+    G = K // 128
+    wg = wf.astype(np.float64).reshape(N, G, 128)
+    Sd = S.astype(np.float64)
+    lo, hi = wg.min(axis=2), wg.max(axis=2)
+    # the scale is (hi - lo)/15 up to one fp32 and one fp16 rounding
+    ratio = (hi - lo) / Sd / 15.0
+    assert np.all(np.abs(ratio - 1) <= 2.0 ** -11 + 2.0 ** -23)
+    # the group minimum lands on code 0 when z is not clamped
+    qg = q.reshape(N, G, 128)
+    argmin = wg.argmin(axis=2)
+    qlo = np.take_along_axis(qg, argmin[..., None], axis=2)[..., 0]
+    unclamped = (-lo / Sd) <= 15.5
+    assert np.all(qlo[unclamped] == 0)
+    # dequantization error <= S/2, except codes clamped at 15 (rounded S), by at most 15 * 2^-11 S
+    what = O.dequantize(q, S, z).reshape(N, G, 128)
+    err = np.abs(what - wg)
+    assert np.all(err <= Sd[..., None] * (0.5 + 0.008))
+    over = err > Sd[..., None] * 0.5 * (1 + 1e-12)
+    assert np.all(qg[over] == 15)
+
+
+# ----------------------------------------------------------------------------
+# dequantization and matmul: exact rational arithmetic
+# ----------------------------------------------------------------------------
+def test_dequantize_exact_rational():
+    rng = np.random.default_rng(5)
+    q = rng.integers(0, 16, (3, 256)).astype(np.uint8)
+    z = rng.integers(0, 16, (3, 2)).astype(np.uint8)
+    S = (rng.uniform(1e-4, 2.0, (3, 2))).astype(np.float16)
+    d = O.dequantize(q, S, z)
+    for n in range(3):
+        for k in range(0, 256, 7):
+            g = k // 128
+            exact = (Fraction(int(q[n, k])) - int(z[n, g])) * Fraction(float(S[n, g]))
+            assert Fraction(float(d[n, k])) == exact
+
+
+def test_linear_matches_exact_rationals():
+    rng = np.random.default_rng(11)
+    for (M, K, N) in [(1, 128, 3), (4, 256, 16), (2, 128, 5)]:
+        xs = rng.standard_normal((M, K)).astype(np.float16)
+        w = rng.standard_normal((N, K)).astype(np.float16).astype(np.float64)
+        y = O.linear(xs, w)
+        assert y.shape == (M, N)
+        for m in range(M):
+            for n in range(N):
+                ex = sum(Fraction(float(xs[m, k])) * Fraction(float(w[n, k])) for k in range(K))
+                assert abs(float(ex) - y[m, n]) <= 1e-12 * max(1.0, abs(float(ex)))
+
+
+# ----------------------------------------------------------------------------
+# activation statistic, activation scaling, fold
+# ----------------------------------------------------------------------------
+def test_activation_scale_closed_forms():
+    x = np.array([[0, 1, 4, -9, 0.5],
+                  [0, -1, 0, -16, 0.5]], dtype=np.float16)
+    s = O.activation_scale(x)
+    expect = [math.sqrt(1e-8), 1.0, math.sqrt(2.0), math.sqrt(12.5), math.sqrt(0.5)]
+    assert s.dtype == np.float32
+    assert s.tolist() == [float(np.float32(e)) for e in expect]
+    # alpha = 1 gives the mean, alpha = 0 gives 1
+    s1 = O.activation_scale(x, alpha=1.0)
+    assert s1.tolist() == [float(np.float32(e)) for e in [1e-8, 1.0, 2.0, 12.5, 0.5]]
+    assert np.all(O.activation_scale(x, alpha=0.0) == 1.0)
+
+
+def test_activation_scale_exact_mean():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((37, 64)) * 30).astype(np.float16)
+    s = O.activation_scale(x, alpha=1.0)
+    for j in range(64):
+        mean = sum(Fraction(abs(float(v))) for v in x[:, j]) / 37
+        assert float(s[j]) == float(np.float32(float(mean)))
+
+
+def test_scale_activations_closed_form():
+    x = np.array([[1.0, -3.0, 0.0]], dtype=np.float16)
+    s = np.array([math.sqrt(2.0), 0.5, 7.0], dtype=np.float32)
+    xs = O.scale_activations(x, s)
+    # 1/1.4142135 = 0.70710677 -> fp16 0.70703125 (0x39a8); -3/0.5 = -6; 0/7 = 0
+    assert _f16_bits(xs)[0].tolist() == [0x39A8, int(_f16_bits(np.float16(-6.0))), 0]
+
+
+def test_fold_direction_equivalence_exact():
+    """(W diag(s)) (diag(1/s) x) = W x, computed exactly, so the fold goes on columns k."""
+    rng = np.random.default_rng(9)
+    M, N, K = 3, 5, 256
+    x, W = workloads.random_case(9, M, N, K)
+    s = O.activation_scale(x)
+    # exact float64 version of both halves of the transform
+    Wd = W.astype(np.float64) * s.astype(np.float64)[None, :]
+    xd = x.astype(np.float64) / s.astype(np.float64)[None, :]
+    lhs = xd @ Wd.T
+    rhs = x.astype(np.float64) @ W.astype(np.float64).T
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12 * np.abs(rhs).max())
+    # the stored (fp16-rounded) halves keep the product to fp16 accuracy
+    y16 = O.scale_activations(x, s).astype(np.float64) @ O.fold_weights(W, s).astype(np.float64).T
+    assert np.linalg.norm(y16 - rhs) / np.linalg.norm(rhs) < 2e-3
+    # the weight side is the one scaled UP on large-activation channels, column by column
+    wf = O.fold_weights(W, s).astype(np.float64)
+    j = int(np.argmax(s))
+    assert s[j] > 2
+    ratio = wf[:, j] / W[:, j].astype(np.float64)
+    assert np.allclose(ratio, s[j], rtol=2e-3)
+    xs = O.scale_activations(x, s).astype(np.float64)
+    assert np.allclose(xs[:, j] * s[j], x[:, j].astype(np.float64), rtol=2e-3)
+
+
+def test_awq_scaling_reduces_error_on_outlier_recipe():
+    """The method's claim: scaling salient (large-activation) channels lowers the output error."""
+    wl = workloads.WORKLOADS["tiny_512"]
+    x, W = workloads.layer_inputs(wl, 0, 1)
+    exact = x.astype(np.float64) @ W.astype(np.float64).T
+    r = O.reference_forward(x, W)
+    plain = O.linear(x, O.fake_quantize(W, None))
+    e_awq = np.linalg.norm(r["y"] - exact) / np.linalg.norm(exact)
+    e_rtn = np.linalg.norm(plain - exact) / np.linalg.norm(exact)
+    assert e_awq < e_rtn
+    assert e_awq < 0.1
+
+
+def test_fold_none_is_identity():
+    _, W = workloads.random_case(2, 1, 7, 128)
+    assert np.array_equal(O.fold_weights(W, None).view(np.uint16), W.view(np.uint16))
+
+
+# ----------------------------------------------------------------------------
+# packed layout
+# ----------------------------------------------------------------------------
+def test_layout_hand_positions():
+    fx = _load("layout_positions.json")
+    N, K = fx["N"], fx["K"]
+    G = K // 128
+    words, nsc, nzb = O.packed_sizes(N, K)
+    assert (words, nsc, nzb) == (fx["sizes"]["words"], fx["sizes"]["scales"], fx["sizes"]["zero_bytes"])
+    for c in fx["codes"]:
+        q = np.zeros((N, K), np.uint8)
+        q[c["n"], c["k"]] = 0xB
+        qw, _, _ = O.pack(q, np.zeros((N, G), np.float16), np.zeros((N, G), np.uint8))
+        nz = np.nonzero(qw)[0]
+        assert nz.tolist() == [c["word"]]
+        assert int(qw[c["word"]]) == 0xB << (4 * c["nibble"])
+    for c in fx["scales"]:
+        S = np.zeros((N, G), np.float16)
+        S[c["n"], c["g"]] = 1.0
+        _, sc, _ = O.pack(np.zeros((N, K), np.uint8), S, np.zeros((N, G), np.uint8))
+        assert np.nonzero(sc)[0].tolist() == [c["index"]]
+    for c in fx["zeros"]:
+        z = np.zeros((N, G), np.uint8)
+        z[c["n"], c["g"]] = 9
+        _, _, zb = O.pack(np.zeros((N, K), np.uint8), np.zeros((N, G), np.float16), z)
+        assert np.nonzero(zb)[0].tolist() == [c["byte"]]
+        assert int(zb[c["byte"]]) == (9 << 4 if c["high"] else 9)
+
+
+@pytest.mark.parametrize("N,K", [(128, 128), (300, 256), (16, 384), (513, 640)])
+def test_layout_roundtrip(N, K):
+    rng = np.random.default_rng(N * 31 + K)
+    G = K // 128
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    S = rng.standard_normal((N, G)).astype(np.float16)
+    z = rng.integers(0, 16, (N, G)).astype(np.uint8)
+    qw, sc, zb = O.pack(q, S, z)
+    assert (qw.size, sc.size, zb.size) == O.packed_sizes(N, K)
+    q2, S2, z2 = O.unpack(qw, sc, zb, N, K)
+    assert np.array_equal(q, q2) and np.array_equal(S.view(np.uint16), S2.view(np.uint16))
+    assert np.array_equal(z, z2)
+    # padding rows decode as zeros
+    Np = O.padded_rows(N)
+    qa, Sa, za = O.unpack(qw, sc, zb, Np, K)
+    assert not qa[N:].any() and not Sa[N:].astype(np.float32).any() and not za[N:].any()
+
+
+def test_layout_lane_chunk_holds_its_fragment():
+    """A lane's 16 bytes (4 words) hold rows r, r+8 and k in [16t, 16t+16) of one 16x64 tile."""
+    N, K = 128, 128
+    G = 1
+    n_idx, k_idx = np.meshgrid(np.arange(N), np.arange(K), indexing="ij")
+    for (nt, r, t, kt) in [(0, 0, 0, 0), (3, 5, 2, 1), (7, 7, 3, 1)]:
+        mark = np.zeros((N, K), np.uint8)
+        rows = [nt * 16 + r, nt * 16 + r + 8]
+        cols = slice(kt * 64 + 16 * t, kt * 64 + 16 * t + 16)
+        mark[rows[0], cols] = 1
+        mark[rows[1], cols] = 1
+        qw, _, _ = O.pack(mark * 15, np.zeros((N, G), np.float16), np.zeros((N, G), np.uint8))
+        lane = 4 * r + t
+        base = (kt * 8 + nt) * 128 + lane * 4
+        assert np.nonzero(qw)[0].tolist() == [base, base + 1, base + 2, base + 3]
+        assert all(int(w) == 0xFFFFFFFF for w in qw[base:base + 4])
+
+
+# ----------------------------------------------------------------------------
+# tolerance check helper and the configuration contract
+# ----------------------------------------------------------------------------
+def test_check_tolerance_boundaries():
+    rng = np.random.default_rng(0)
+    y = rng.standard_normal((4, 64))
+    ok, ef, em = O.check_tolerance(y, y)
+    assert ok and ef == 0 and em == 0
+    rms = np.sqrt(np.mean(y ** 2))
+    bump = y.copy()
+    bump[0, 0] += 0.011 * rms          # max error just above 1e-2 rms
+    assert not O.check_tolerance(bump, y)[0]
+    bump[0, 0] = y[0, 0] + 0.009 * rms
+    assert O.check_tolerance(bump, y)[0]
+    assert not O.check_tolerance(y * (1 + 3e-3), y)[0]    # Frobenius 3e-3
+
+
+def test_quant_config_fixture_is_the_built_configuration():
+    fx = _load("quant_configs.json")
+    hf = fx["hf_quantization_config"]
+    assert (hf["bits"], hf["group_size"], hf["zero_point"]) == (O.BITS, O.GROUP_SIZE, True)
+    aw = fx["autoawq_quant_config"]
+    assert (aw["w_bit"], aw["q_group_size"], aw["zero_point"]) == (O.BITS, O.GROUP_SIZE, True)
+    assert O.QMAX == 2 ** O.BITS - 1
+
+
+def test_reference_forward_tiny_workload_shapes():
+    wl = workloads.WORKLOADS["tiny_512"]
+    x, W = workloads.layer_inputs(wl, 0, 1)
+    r = O.reference_forward(x, W)
+    assert r["q"].shape == (512, 512) and r["S"].shape == (512, 4) and r["y"].shape == (1, 512)
+    assert workloads.n_outlier_channels(512) == 5
