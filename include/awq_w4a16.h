@@ -1,0 +1,180 @@
+/*
+ * awq_w4a16.h — C ABI of the AWQ W4A16 g128 library for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are web pages, cited by title and section):
+ *
+ *   "AWQ: Activation-aware Weight Quantization for LLM Compression and
+ *   Acceleration" (llm-awq README mirror), "Usage" steps 1-3 and
+ *   "Installation" step 3: 4-bit weights quantized in groups of 128 along the
+ *   input dimension, 16-bit activations, CUDA kernels for the context (GEMM)
+ *   and decode (GEMV) stages.
+ *   "transformers - AWQ" (HF guide translation), section 2: the
+ *   quantization_config {quant_method: awq, zero_point: true, group_size: 128,
+ *   bits: 4, version: gemm}.
+ *   CSDN VPTQ blog, section "02.02 AWQ": salient input channels are found
+ *   from activation statistics and protected by scaling them up through an
+ *   equivalent transform (weights times s, activations divided by s).
+ *
+ * Steps of the path and their entry points:
+ *   a1  awq_activation_scale  s_k = max(mean_m |x_mk|, 1e-8)^alpha;  x'_mk = fp16(x_mk / s_k)
+ *       awq_scale_activations x'_mk = fp16(x_mk / s_k) with a stored s
+ *   a2  awq_quantize_g128     w'_nk = fp16(W_nk * s_k); per group of 128 k:
+ *                             S = fp16(max(hi-lo, 1e-5)/15), z = clamp(rint(-lo/S), 0, 15),
+ *                             q = clamp(rint(w'/S) + z, 0, 15)      (fp32, round half to even)
+ *   a3  awq_w4a16_gemv        y[M,N] = x'[M,K] . ((q - z) * S)^T, M <= 32  (fp32 accumulate, fp16 out)
+ *   a4  awq_w4a16_gemm        the same for any M (tensor-core prefill kernel)
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller. The library
+ *     allocates no memory and never synchronizes, except awq_poll_device_status
+ *     and awq_debug_set_wait_budget_ns, which say so.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and runs asynchronously; outputs are valid once the stream reaches
+ *     that point.
+ *   - Arguments are checked on the host before anything is launched. A bad
+ *     argument returns an error code and launches nothing. No call aborts the
+ *     process or throws.
+ *   - fp16 buffers hold IEEE binary16 bit patterns (uint16_t here).
+ *   - Outputs must not alias inputs.
+ *   - Only device ordinals with compute capability 10.0 are supported
+ *     (AWQ_ERR_UNSUPPORTED otherwise).
+ *
+ * Packed layout, version 1 (awq_layout_version() == 1).
+ *   Rows are padded to Np = ceil(N/128)*128 (padding rows: code 0, scale 0,
+ *   zero 0). With
+ *     n = st*128 + nt*16 + h*8 + r        (st super-tile, nt 16-row tile, h half, r row)
+ *     k = kt*64 + t*16 + s*4 + e1*2 + e0  (kt 64-k tile, t column block, s step, e slot)
+ *     g = k / 128,  KT = K/64,  G = K/128
+ *   qweight: uint32[Np*K/8];  code q[n][k] sits in word
+ *            ((st*KT + kt)*8 + nt)*128 + (4*r + t)*4 + s,  nibble h + 2*e1 + 4*e0
+ *            (bits 4*nibble .. 4*nibble+3).  The 16 bytes of words
+ *            (.., 4r+t, 0..3) are exactly the m16n8k16 A-fragments of one lane
+ *            (rows r, r+8; k in [16t, 16t+16) of a 64-k tile).
+ *   scales:  fp16[Np*K/128]; S[n][g] at ((st*G + g)*8 + nt)*16 + 2*r + h
+ *   zeros:   uint8[Np*K/256]; z[n][g] in byte ((st*G + g)*8 + nt)*8 + r,
+ *            low nibble for h = 0, high nibble for h = 1.
+ *   Base pointers of qweight, scales, zeros, x, x' and y must be 16-byte aligned.
+ */
+#ifndef AWQ_W4A16_H_
+#define AWQ_W4A16_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define AWQ_API __attribute__((visibility("default")))
+#else
+#define AWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                      /* the same type cudaStream_t points to */
+typedef struct CUstream_st* awq_stream_t;
+
+typedef enum {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, size out of range */
+  AWQ_ERR_UNSUPPORTED = 2,   /* configuration or device not built (bits != 4, group != 128, ...) */
+  AWQ_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+  AWQ_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  AWQ_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (reported by awq_poll_device_status) */
+} awq_status_t;
+
+/* Packed-layout version; bumps whenever the layout above changes. */
+AWQ_API int awq_layout_version(void);
+
+/* Static, human-readable name of a status code. Never NULL. */
+AWQ_API const char* awq_status_string(int status);
+
+/* AWQ_OK iff (bits, group_size, zero_point) is the built configuration
+ * (4, 128, 1) — the quantization_config of "transformers - AWQ" section 2 and
+ * the quant_config of the AutoAWQ section of the llmstudio.ru page.
+ * AWQ_ERR_UNSUPPORTED otherwise. Pure host function. */
+AWQ_API awq_status_t awq_check_config(int bits, int group_size, int zero_point);
+
+/* Sizes in bytes of the packed arrays for an N x K layer (0 if N < 1,
+ * K < 128 or K % 128 != 0). Pure host functions. */
+AWQ_API size_t awq_qweight_bytes(int N, int K);
+AWQ_API size_t awq_scales_bytes(int N, int K);
+AWQ_API size_t awq_zeros_bytes(int N, int K);
+
+/* a1. Activation statistic and activation scaling (CSDN blog "02.02 AWQ":
+ * scales from activation statistics; equivalent transform).
+ *   x        fp16 [M, K] row-major (device).
+ *   s_out    fp32 [K] (device): s_k = max(mean_m |x_mk|, 1e-8)^alpha, computed in
+ *            float64 (the column sum is exact: integers in units of 2^-24) and
+ *            rounded to fp32; alpha = 0.5 uses the correctly rounded square root.
+ *   x_scaled fp16 [M, K] (device) or NULL: x'_mk = fp16_rn(fp32(x_mk) / s_k)
+ *            (IEEE fp32 division).
+ * Requires 1 <= M, 1 <= K, K % 8 == 0. alpha must be finite. */
+AWQ_API awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha,
+                                  float* s_out, uint16_t* x_scaled, awq_stream_t stream);
+
+/* a1 (inference form). x'_mk = fp16_rn(fp32(x_mk) / s_k) with a stored s
+ * (calibrated once by awq_activation_scale); the activation half of the
+ * equivalent transform of CSDN "02.02 AWQ".
+ *   x        fp16 [M, K] row-major (device);  s  fp32 [K] (device, 16-byte aligned)
+ *   x_scaled fp16 [M, K] (device).
+ * Bit-identical to the x_scaled output of awq_activation_scale for the same s.
+ * Requires 1 <= M, 1 <= K, K % 8 == 0. */
+AWQ_API awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int K, uint16_t* x_scaled,
+                                   awq_stream_t stream);
+
+/* a2. Fold + asymmetric 4-bit group quantizer, group size 128 along K
+ * ("Usage" steps 1-3 of the llm-awq README: --w_bit 4 --q_group_size 128,
+ * --q_backend real; HF config zero_point true).
+ *   W          fp16 [N, K] row-major (device).
+ *   fold_scale fp32 [K] (device) or NULL (= all ones, no fold).
+ *   qweight, scales, zeros: outputs in packed layout v1, sizes from awq_*_bytes.
+ * Codes, scales and zeros are bit-identical to the rules in the file header
+ * (every step IEEE fp32, round to nearest even). Requires N >= 1, K >= 128,
+ * K % 128 == 0. Values with |W*s| >= 65520 overflow fp16 to inf; the result is
+ * then defined by the same IEEE rules but is not a useful quantization. */
+AWQ_API awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K,
+                               uint32_t* qweight, uint16_t* scales, uint8_t* zeros,
+                               awq_stream_t stream);
+
+/* a3. Decode W4A16 linear layer (context: "Installation" step 3 of the llm-awq
+ * README, W4A16 decode kernels).
+ *   x  fp16 [M, K] row-major (the scaled activations x'), 1 <= M <= 32.
+ *   y  fp16 [M, N] row-major.
+ * y = x . dequant^T with fp32 accumulation; dequant(q) = (q - z) * S.
+ * Requires N >= 1, K >= 128, K % 128 == 0. */
+AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                            const uint8_t* zeros, uint16_t* y, int M, int N, int K,
+                            awq_stream_t stream);
+
+/* a4. Prefill W4A16 linear layer (tcgen05 tensor cores, TMEM accumulators,
+ * TMA-fed pipeline). Same arguments and result as awq_w4a16_gemv, any M >= 1
+ * (M <= 2^31-1 / K). Weights are dequantized to fp16 ((q - z) * S rounded
+ * once) before the fp16 x fp16 -> fp32 tensor-core products. */
+AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                            const uint8_t* zeros, uint16_t* y, int M, int N, int K,
+                            awq_stream_t stream);
+
+/* Convenience dispatch: awq_w4a16_gemv for M <= 32, awq_w4a16_gemm otherwise. */
+AWQ_API awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                              const uint8_t* zeros, uint16_t* y, int M, int N, int K,
+                              awq_stream_t stream);
+
+/* Synchronizes `stream`, then reads and clears the device status word of the
+ * current device. Returns AWQ_ERR_TIMEOUT if a kernel since the last poll gave
+ * up a bounded wait (its outputs are then undefined), AWQ_ERR_CUDA if the
+ * stream reports an error, AWQ_OK otherwise. */
+AWQ_API awq_status_t awq_poll_device_status(awq_stream_t stream);
+
+/* Test hook: sets the time (ns) after which a bounded wait inside a kernel
+ * gives up on the current device (0 restores the default of 2 s). Synchronous.
+ * A kernel that gives up sets the status read by awq_poll_device_status,
+ * drains its own copies and tensor-core work in flight, frees its tensor
+ * memory and returns. */
+AWQ_API awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* AWQ_W4A16_H_ */

@@ -1,0 +1,113 @@
+"""The C-ABI library: it builds, loads and exports every declared symbol; host-only logic.
+
+No test here calls into CUDA: argument checks that fail return before the
+library touches the device, and only those paths are exercised.
+"""
+import ctypes
+import json
+import os
+import re
+import subprocess
+
+import pytest
+
+from oracle import awq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq_w4a16.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from weight_only_quantization_w4a16_b200 import build as B
+    import weight_only_quantization_w4a16_b200 as P
+    B.build()
+    return P.load_library()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^AWQ_API [^(]*?\b(awq_\w+)\(", src, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for n in ["awq_activation_scale", "awq_scale_activations", "awq_quantize_g128", "awq_w4a16_gemv",
+              "awq_w4a16_gemm", "awq_w4a16_linear", "awq_poll_device_status", "awq_layout_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import weight_only_quantization_w4a16_b200 as P
+    out = subprocess.run(["nm", "-D", "--defined-only", P.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (awq_\w+)$", out, flags=re.M))
+    declared = set(_declared())
+    assert declared <= exported, declared - exported
+    # nothing else leaks out of the library (static cudart stays internal)
+    assert all(name.startswith("awq_") for name in re.findall(r" [TDBRW] (\S+)$", out, flags=re.M))
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_layout_version_and_status_strings(lib):
+    assert lib.awq_layout_version() == 1
+    for code in range(6):
+        s = lib.awq_status_string(code).decode()
+        assert s.startswith("AWQ_")
+    assert lib.awq_status_string(99).decode() == "AWQ_ERR_UNKNOWN"
+
+
+def test_check_config_against_page_configs(lib):
+    fx = json.load(open(os.path.join(ROOT, "tests", "golden", "quant_configs.json")))
+    hf = fx["hf_quantization_config"]
+    assert lib.awq_check_config(hf["bits"], hf["group_size"], int(hf["zero_point"])) == 0
+    aw = fx["autoawq_quant_config"]
+    assert lib.awq_check_config(aw["w_bit"], aw["q_group_size"], int(aw["zero_point"])) == 0
+    for u in fx["unsupported_examples"]:
+        assert lib.awq_check_config(u["bits"], u["group_size"], int(u["zero_point"])) == 2
+
+
+@pytest.mark.parametrize("N,K", [(1, 128), (128, 128), (300, 256), (4096, 11008), (28672, 8192), (513, 640)])
+def test_packed_sizes_match_layout_spec(lib, N, K):
+    words, sc, zb = O.packed_sizes(N, K)
+    assert lib.awq_qweight_bytes(N, K) == 4 * words
+    assert lib.awq_scales_bytes(N, K) == 2 * sc
+    assert lib.awq_zeros_bytes(N, K) == zb
+
+
+@pytest.mark.parametrize("N,K", [(0, 128), (16, 0), (16, 100), (16, 192), (-1, 128)])
+def test_packed_sizes_reject_bad_shapes(lib, N, K):
+    assert lib.awq_qweight_bytes(N, K) == 0 and lib.awq_scales_bytes(N, K) == 0 and lib.awq_zeros_bytes(N, K) == 0
+
+
+A = 0x10000   # aligned fake addresses: never dereferenced, every call below fails its checks first
+MIS = 0x10008
+
+
+def test_argument_checks_fail_before_any_device_call(lib):
+    V = ctypes.c_void_p
+    # null pointers
+    assert lib.awq_quantize_g128(None, None, 16, 128, V(A), V(A), V(A), None) == 1
+    assert lib.awq_w4a16_gemv(V(A), V(A), V(A), None, V(A), 1, 16, 128, None) == 1
+    assert lib.awq_w4a16_gemm(None, V(A), V(A), V(A), V(A), 1, 16, 128, None) == 1
+    assert lib.awq_activation_scale(None, 1, 128, 0.5, V(A), None, None) == 1
+    assert lib.awq_scale_activations(V(A), None, 1, 128, V(A), None) == 1
+    # bad sizes
+    assert lib.awq_quantize_g128(V(A), None, 16, 100, V(A), V(A), V(A), None) == 1
+    assert lib.awq_quantize_g128(V(A), None, 0, 128, V(A), V(A), V(A), None) == 1
+    assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(A), 33, 16, 128, None) == 1
+    assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(A), 0, 16, 128, None) == 1
+    assert lib.awq_w4a16_gemm(V(A), V(A), V(A), V(A), V(A), 4, 16, 192, None) == 1
+    assert lib.awq_activation_scale(V(A), 1, 12, 0.5, V(A), None, None) == 1
+    assert lib.awq_activation_scale(V(A), 1, 128, float("nan"), V(A), None, None) == 1
+    # misaligned pointers
+    assert lib.awq_quantize_g128(V(MIS), None, 16, 128, V(A), V(A), V(A), None) == 3
+    assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(MIS), 1, 16, 128, None) == 3
+    assert lib.awq_w4a16_gemm(V(A), V(MIS), V(A), V(A), V(A), 300, 16, 128, None) == 3
+    assert lib.awq_scale_activations(V(A), V(MIS), 1, 128, V(A), None) == 3
+
+
+def test_binding_refuses_to_run_without_library(tmp_path):
+    import weight_only_quantization_w4a16_b200 as P
+    with pytest.raises(RuntimeError, match="no fallback"):
+        P.load_library(str(tmp_path / "missing.so"))

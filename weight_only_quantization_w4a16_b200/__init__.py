@@ -1,0 +1,270 @@
+"""AWQ W4A16 g128 for NVIDIA B200 — Python binding of ``libawq_w4a16.so``.
+
+The binding only marshals arguments: it checks tensor dtypes, shapes and
+devices, allocates outputs with PyTorch when the caller gives none, and
+passes raw device pointers plus the current CUDA stream to the C ABI declared
+in ``include/awq_w4a16.h``. Every step of the path runs in the library's
+CUDA kernels; if the library is missing, every call raises.
+
+Functions (same names as the C ABI):
+
+* ``awq_activation_scale(x, alpha)``  -> (s[K] fp32, x'[M,K] fp16)
+* ``awq_scale_activations(x, s)`` -> x'[M,K] fp16 with a stored s
+* ``awq_quantize_g128(W, fold_scale)`` -> (qweight int32, scales fp16, zeros uint8)
+* ``awq_w4a16_gemv(x, qweight, scales, zeros, N)`` -> y[M,N] fp16 (M <= 32)
+* ``awq_w4a16_gemm(x, qweight, scales, zeros, N)`` -> y[M,N] fp16
+* ``awq_w4a16_linear(...)``: gemv for M <= 32, gemm otherwise
+* ``awq_poll_device_status()``, ``awq_debug_set_wait_budget_ns(ns)``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libawq_w4a16.so")
+
+AWQ_OK = 0
+AWQ_ERR_INVALID_ARG = 1
+AWQ_ERR_UNSUPPORTED = 2
+AWQ_ERR_MISALIGNED = 3
+AWQ_ERR_CUDA = 4
+AWQ_ERR_TIMEOUT = 5
+
+GROUP_SIZE = 128
+BITS = 4
+
+_lib = None
+
+
+class AWQError(RuntimeError):
+    """A C-ABI call returned a status other than AWQ_OK."""
+
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg}")
+        self.status = status
+
+
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGS = {
+    "awq_layout_version": ([], ctypes.c_int),
+    "awq_status_string": ([_I], ctypes.c_char_p),
+    "awq_check_config": ([_I, _I, _I], _I),
+    "awq_qweight_bytes": ([_I, _I], ctypes.c_size_t),
+    "awq_scales_bytes": ([_I, _I], ctypes.c_size_t),
+    "awq_zeros_bytes": ([_I, _I], ctypes.c_size_t),
+    "awq_activation_scale": ([_VP, _I, _I, ctypes.c_float, _VP, _VP, _VP], _I),
+    "awq_scale_activations": ([_VP, _VP, _I, _I, _VP, _VP], _I),
+    "awq_quantize_g128": ([_VP, _VP, _I, _I, _VP, _VP, _VP, _VP], _I),
+    "awq_w4a16_gemv": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
+    "awq_w4a16_gemm": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
+    "awq_w4a16_linear": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
+    "awq_poll_device_status": ([_VP], _I),
+    "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
+}
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library(path: Optional[str] = None):
+    """Loads libawq_w4a16.so (built in-tree by ``build.py``). Raises if absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(
+            f"{p} is missing: build it with `python -m weight_only_quantization_w4a16_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(p)
+    for name, (args, res) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().awq_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != AWQ_OK:
+        raise AWQError(fn, status, status_string(status))
+
+
+def layout_version() -> int:
+    return int(load_library().awq_layout_version())
+
+
+def check_config(bits: int, group_size: int, zero_point: bool) -> bool:
+    return load_library().awq_check_config(int(bits), int(group_size), int(bool(zero_point))) == AWQ_OK
+
+
+def packed_nbytes(N: int, K: int) -> Tuple[int, int, int]:
+    lib = load_library()
+    return (int(lib.awq_qweight_bytes(N, K)), int(lib.awq_scales_bytes(N, K)), int(lib.awq_zeros_bytes(N, K)))
+
+
+# ---------------------------------------------------------------------------- torch marshalling
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr():
+    torch = _torch()
+    return _VP(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t) -> _VP:
+    return _VP(t.data_ptr()) if t is not None else _VP(0)
+
+
+def _need(t, dtype, name, dims=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions")
+
+
+def awq_activation_scale(x, alpha: float = 0.5, s_out=None, x_scaled=None, want_scaled: bool = True):
+    """a1: s[K] = max(mean_m |x[m,k]|, 1e-8)^alpha and x' = fp16(x / s)."""
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    M, K = x.shape
+    if s_out is None:
+        s_out = torch.empty(K, dtype=torch.float32, device=x.device)
+    _need(s_out, torch.float32, "s_out", 1)
+    if want_scaled and x_scaled is None:
+        x_scaled = torch.empty_like(x)
+    if x_scaled is not None:
+        _need(x_scaled, torch.float16, "x_scaled", 2)
+    st = load_library().awq_activation_scale(_ptr(x), M, K, float(alpha), _ptr(s_out), _ptr(x_scaled),
+                                             _stream_ptr())
+    _check("awq_activation_scale", st)
+    return s_out, x_scaled
+
+
+def alloc_packed(N: int, K: int, device="cuda"):
+    """Output tensors for awq_quantize_g128: qweight (int32 words), scales (fp16), zeros (uint8)."""
+    torch = _torch()
+    qb, sb, zb = packed_nbytes(N, K)
+    if qb == 0:
+        raise ValueError("N >= 1 and K a positive multiple of 128 are required")
+    return (torch.empty(qb // 4, dtype=torch.int32, device=device),
+            torch.empty(sb // 2, dtype=torch.float16, device=device),
+            torch.empty(zb, dtype=torch.uint8, device=device))
+
+
+def awq_quantize_g128(W, fold_scale=None, out=None):
+    """a2: fold s into W[N,K] and quantize to packed layout v1. Returns (qweight, scales, zeros)."""
+    torch = _torch()
+    _need(W, torch.float16, "W", 2)
+    N, K = W.shape
+    if fold_scale is not None:
+        _need(fold_scale, torch.float32, "fold_scale", 1)
+    qweight, scales, zeros = out if out is not None else alloc_packed(N, K, W.device)
+    _need(qweight, torch.int32, "qweight")
+    _need(scales, torch.float16, "scales")
+    _need(zeros, torch.uint8, "zeros")
+    st = load_library().awq_quantize_g128(_ptr(W), _ptr(fold_scale), N, K, _ptr(qweight), _ptr(scales),
+                                          _ptr(zeros), _stream_ptr())
+    _check("awq_quantize_g128", st)
+    return qweight, scales, zeros
+
+
+def _linear(fn_name: str, x, qweight, scales, zeros, N: int, y=None):
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    _need(qweight, torch.int32, "qweight")
+    _need(scales, torch.float16, "scales")
+    _need(zeros, torch.uint8, "zeros")
+    M, K = x.shape
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _need(y, torch.float16, "y", 2)
+    if tuple(y.shape) != (M, N):
+        raise ValueError("y must have shape (M, N)")
+    qb, sb, zb = packed_nbytes(N, K)
+    if qweight.numel() * 4 < qb or scales.numel() * 2 < sb or zeros.numel() < zb:
+        raise ValueError("packed weight tensors are too small for (N, K)")
+    st = getattr(load_library(), fn_name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K,
+                                          _stream_ptr())
+    _check(fn_name, st)
+    return y
+
+
+def awq_w4a16_gemv(x, qweight, scales, zeros, N: int, y=None):
+    """a3: y[M,N] = x' . dequant^T for M <= 32 (decode)."""
+    return _linear("awq_w4a16_gemv", x, qweight, scales, zeros, N, y)
+
+
+def awq_w4a16_gemm(x, qweight, scales, zeros, N: int, y=None):
+    """a4: y[M,N] = x' . dequant^T on tcgen05 tensor cores (prefill)."""
+    return _linear("awq_w4a16_gemm", x, qweight, scales, zeros, N, y)
+
+
+def awq_w4a16_linear(x, qweight, scales, zeros, N: int, y=None):
+    """gemv for M <= 32, gemm otherwise."""
+    return _linear("awq_w4a16_linear", x, qweight, scales, zeros, N, y)
+
+
+def awq_poll_device_status() -> int:
+    """Synchronizes the current stream and returns (and clears) the device status code."""
+    return int(load_library().awq_poll_device_status(_stream_ptr()))
+
+
+def awq_debug_set_wait_budget_ns(ns: int) -> None:
+    _check("awq_debug_set_wait_budget_ns", load_library().awq_debug_set_wait_budget_ns(int(ns)))
+
+
+class AWQLinear:
+    """A quantized linear layer: packed weights plus the per-channel fold scale.
+
+    ``AWQLinear.from_float(W, x_calib)`` runs the whole path on the GPU: the
+    activation statistic of ``x_calib`` (a1), the fold and quantizer (a2);
+    ``layer(x)`` scales the activations by 1/s and runs the W4A16 kernel
+    (a3 for M <= 32, a4 otherwise).
+    """
+
+    def __init__(self, qweight, scales, zeros, s, N: int, K: int):
+        self.qweight, self.scales, self.zeros, self.s = qweight, scales, zeros, s
+        self.N, self.K = N, K
+
+    @classmethod
+    def from_float(cls, W, x_calib, alpha: float = 0.5):
+        s, _ = awq_activation_scale(x_calib, alpha, want_scaled=False)
+        q, sc, z = awq_quantize_g128(W, s)
+        return cls(q, sc, z, s, W.shape[0], W.shape[1])
+
+    def __call__(self, x, y=None):
+        xs = awq_scale_activations(x, self.s)
+        return awq_w4a16_linear(xs, self.qweight, self.scales, self.zeros, self.N, y)
+
+
+def awq_scale_activations(x, s, x_scaled=None):
+    """a1 with a stored s: x' = fp16(x / s) (the activation half of the equivalent transform)."""
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    _need(s, torch.float32, "s", 1)
+    M, K = x.shape
+    if x_scaled is None:
+        x_scaled = torch.empty_like(x)
+    _need(x_scaled, torch.float16, "x_scaled", 2)
+    st = load_library().awq_scale_activations(_ptr(x), _ptr(s), M, K, _ptr(x_scaled), _stream_ptr())
+    _check("awq_scale_activations", st)
+    return x_scaled

@@ -1,0 +1,266 @@
+// awq_gemm.cuh — a4: prefill W4A16 linear layer on tcgen05 tensor cores.
+//
+// llm-awq README, "Installation" step 3 (W4A16 kernels for the context
+// stage) and HF "transformers - AWQ" section 2 ("version": "gemm").
+// y[M,N] = x'[M,K] . ((q-z)*S)^T with fp16 operands and fp32 accumulation.
+//
+// The contraction runs "swapped": the dequantized weight tile is the MMA's
+// 128-row A operand (one 128-row super-tile of the packed layout), and a
+// tile of BT tokens of x' is the B operand, so every dequantized weight feeds
+// BT tokens. Per CTA (persistent, one per SM):
+//   warp NDQ+4 (one lane): producer — 1-D bulk copies of the packed codes
+//       (4 KB), scales (256 B) and zeros (64 B) of a (super-tile, 64-k) block
+//       and a 2-D TMA load of the x' tile (BT x 64, 128-byte swizzle) into a
+//       STAGES-deep shared-memory ring (mbarrier transaction counts);
+//   warps 0..NDQ-1: dequantize codes to fp16 (q - z) * S straight into the
+//       A tile in the canonical K-major 128-byte-swizzle layout (bank-conflict
+//       free 8-byte stores), then fence.proxy.async and arrive;
+//   warp NDQ+5 (one lane): issues tcgen05.mma kind::f16 128 x BT x 16 into a
+//       TMEM accumulator, commits each stage back to the producer;
+//   warps NDQ..NDQ+3: epilogue — tcgen05.ld of the accumulator (each warp its
+//       32-lane quarter), fp16 convert, coalesced stores of y; two TMEM
+//       accumulators let the epilogue of one tile overlap the next mainloop.
+// Every mbarrier wait is bounded by %globaltimer; on expiry the CTA records
+// AWQ_ERR_TIMEOUT in the device status word, every role stops, the producer
+// waits for its copies in flight, the MMA thread for its MMAs, and TMEM is
+// freed before the CTA returns.
+#pragma once
+
+#include "awq_common.cuh"
+
+namespace awq {
+
+template <int BT, int STAGES, int NDQ>
+struct GemmCfg {
+  static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
+  static_assert(NDQ == 4 || NDQ == 8, "dequant warps");
+  static constexpr int kA = kSuperRows * kKTile * 2;        // 16 KB dequantized weights
+  static constexpr int kB = BT * kKTile * 2;                // x' tile
+  static constexpr int kRawQ = kSuperChunkWords * 4;        // 4096 B
+  static constexpr int kRawS = 8 * 16 * 2;                  // 256 B
+  static constexpr int kRawZ = 8 * 8;                       // 64 B
+  static constexpr int kTx = kB + kRawQ + kRawS + kRawZ;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + STAGES * kA;
+  static constexpr int kOffQ = kOffB + STAGES * kB;
+  static constexpr int kOffS = kOffQ + STAGES * kRawQ;
+  static constexpr int kOffZ = kOffS + STAGES * kRawS;
+  static constexpr int kOffBar = (kOffZ + STAGES * kRawZ + 15) / 16 * 16;
+  // barriers: full[S], aready[S], empty[S], accfull[2], accempty[2], drain[1]
+  static constexpr int kNumBars = 3 * STAGES + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffMisc + 16 + 1024;        // + slack for 1024-byte alignment
+  static constexpr int kTmemCols = 2 * BT < 32 ? 32 : 2 * BT;
+  static constexpr int kThreads = (NDQ + 6) * 32;
+  static constexpr int kWarpEpi0 = NDQ;
+  static constexpr int kWarpProd = NDQ + 4;
+  static constexpr int kWarpMma = NDQ + 5;
+  static_assert(kSmem <= 232448, "shared memory");
+};
+
+template <int BT, int STAGES, int NDQ>
+__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ>::kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
+                const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
+                int N, int K) {
+  using C = GemmCfg<BT, STAGES, NDQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* aready = bars + STAGES;
+  uint64_t* empty = bars + 2 * STAGES;
+  uint64_t* accfull = bars + 3 * STAGES;
+  uint64_t* accempty = accfull + 2;
+  uint64_t* drain = accfull + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NST = padded_rows(N) / kSuperRows;
+  const int MTT = (M + BT - 1) / BT;
+  const int ntiles = NST * MTT;
+  const int KB = K / kKTile;
+  const int G = K / kGroup;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&aready[s], NDQ);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == C::kWarpProd && lane == 0) tma_prefetch_desc(&tmap_x);
+  if (warp == C::kWarpMma) {
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const unsigned long long budget = g_wait_budget_ns;
+
+  if (warp == C::kWarpProd) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_par = 0;   // per stage: loaded at least once / parity of last load
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int st = tile % NST, mt = tile / NST;
+        const uint32_t* qsrc = qweight + static_cast<size_t>(st) * KB * kSuperChunkWords;
+        const __half* ssrc = scales + static_cast<size_t>(st) * G * 128;
+        const uint8_t* zsrc = zeros + static_cast<size_t>(st) * G * 64;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::kTx);
+          bulk_g2s(smem + C::kOffQ + stage * C::kRawQ, qsrc + static_cast<size_t>(kb) * kSuperChunkWords, C::kRawQ,
+                   &full[stage]);
+          bulk_g2s(smem + C::kOffS + stage * C::kRawS, ssrc + static_cast<size_t>(kb >> 1) * 128, C::kRawS,
+                   &full[stage]);
+          bulk_g2s(smem + C::kOffZ + stage * C::kRawZ, zsrc + static_cast<size_t>(kb >> 1) * 64, C::kRawZ,
+                   &full[stage]);
+          tma_load_2d(smem + C::kOffB + stage * C::kB, &tmap_x, kb * kKTile, mt * BT, &full[stage]);
+          issued_mask |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // drain: every copy this thread issued has landed before the CTA may exit
+      int never = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s))
+          mbar_wait_bounded(&full[s], (last_par >> s) & 1u, &never, kDrainBudgetNs);
+    }
+  } else if (warp == C::kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(kSuperRows, BT);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any = false;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+        const int b = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!mbar_wait_bounded(&accempty[b], (use & 1) ^ 1, s_abort, budget)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BT);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget) ||
+              !mbar_wait_bounded(&aready[stage], phase, s_abort, budget)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + C::kOffA + stage * C::kA);
+          const uint32_t b0 = smem_u32(smem + C::kOffB + stage * C::kB);
+#pragma unroll
+          for (int kk = 0; kk < kKTile / 16; ++kk)
+            tc_mma_f16(d_tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), idesc,
+                       (kb | kk) != 0 ? 1u : 0u);
+          any = true;
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(&accfull[b]);
+      }
+      if (any) {
+        int never = 0;
+        tc_commit(drain);
+        mbar_wait_bounded(drain, 0, &never, kDrainBudgetNs);
+      }
+    }
+  } else if (warp < NDQ) {
+    // ------------------------------------------------------------ dequantize
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget)) { ok = false; break; }
+        const uint32_t* rq = reinterpret_cast<const uint32_t*>(smem + C::kOffQ + stage * C::kRawQ);
+        const uint32_t* rs = reinterpret_cast<const uint32_t*>(smem + C::kOffS + stage * C::kRawS);
+        const uint8_t* rz = smem + C::kOffZ + stage * C::kRawZ;
+        uint8_t* A = smem + C::kOffA + stage * C::kA;
+#pragma unroll
+        for (int u = 0; u < 8 / NDQ; ++u) {
+          const int c = warp * 32 + lane + u * 32 * NDQ;   // (16-row tile, lane) chunk
+          const int nt = c >> 5, lw = c & 31, r = lw >> 2, t = lw & 3;
+          const uint4 words = *reinterpret_cast<const uint4*>(rq + nt * kChunkWords + lw * 4);
+          const uint32_t sp = rs[nt * 8 + r];                        // (S_r, S_{r+8})
+          const uint32_t zb = rz[nt * 8 + r];
+          const uint32_t s_r = __byte_perm(sp, 0, 0x1010);          // (S_r, S_r)
+          const uint32_t s_r8 = __byte_perm(sp, 0, 0x3232);         // (S_{r+8}, S_{r+8})
+          const uint32_t za = 0x64006400u | ((zb & 0xFu) * 0x00010001u);
+          const uint32_t zc = 0x64006400u | ((zb >> 4) * 0x00010001u);
+          uint8_t* rowA = A + (nt * 16 + r) * 128;
+          uint8_t* rowB = rowA + 8 * 128;
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) {
+            const int s = ii ^ ((r >> 1) & 1);                      // rotation keeps 8-byte stores conflict free
+            const uint32_t q = (s == 0) ? words.x : (s == 1) ? words.y : (s == 2) ? words.z : words.w;
+            const uint32_t p0 = hmul2_u32(hsub2_u32(lop_or(q, 0x000F000Fu, 0x64006400u), za), s_r);
+            const uint32_t p1 = hmul2_u32(hsub2_u32(lop_or(q >> 4, 0x000F000Fu, 0x64006400u), zc), s_r8);
+            const uint32_t p2 = hmul2_u32(hsub2_u32(lop_or(q >> 8, 0x000F000Fu, 0x64006400u), za), s_r);
+            const uint32_t p3 = hmul2_u32(hsub2_u32(lop_or(q >> 12, 0x000F000Fu, 0x64006400u), zc), s_r8);
+            const int off = (((2 * t + (s >> 1)) ^ r) << 4) + (s & 1) * 8;
+            *reinterpret_cast<uint2*>(rowA + off) = make_uint2(p0, p2);
+            *reinterpret_cast<uint2*>(rowB + off) = make_uint2(p1, p3);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&aready[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - C::kWarpEpi0;   // == warp % 4: TMEM lane quarter of this warp
+    bool ok = true;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      const int st = tile % NST, mt = tile / NST;
+      const int b = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      if (!mbar_wait_bounded(&accfull[b], use & 1, s_abort, budget)) { ok = false; break; }
+      tc_fence_after();
+      const int n = st * kSuperRows + 32 * e + lane;
+      const bool n_ok = n < N;
+#pragma unroll 1
+      for (int cc = 0; cc < BT / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * e) << 16) + static_cast<uint32_t>(b * BT + 32 * cc), v);
+        tc_wait_ld();
+        const int mb = mt * BT + 32 * cc;
+        if (n_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int m = mb + j;
+            if (m < M) y[static_cast<size_t>(m) * N + n] = __float2half_rn(__uint_as_float(v[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+}  // namespace awq

@@ -1,0 +1,340 @@
+// awq_lib.cu — the C ABI of libawq_w4a16 (declared in include/awq_w4a16.h).
+//
+// Host side only: argument checks, launch configuration, TMA descriptors and
+// the device status word. Every step of the path runs in the kernels
+// included below; there is no host or CPU fallback.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "awq_act.cuh"
+#include "awq_common.cuh"
+#include "awq_gemm.cuh"
+#include "awq_gemv.cuh"
+#include "awq_quant.cuh"
+#include "awq_w4a16.h"
+
+namespace awq {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::atomic<int> state{0};   // 0 unknown, 1 supported, 2 unsupported
+  int num_sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device, checked to be compute capability 10.0 (B200 / sm_100a).
+awq_status_t current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return AWQ_ERR_UNSUPPORTED;
+  DeviceInfo& d = g_devices[dev];
+  int st = d.state.load(std::memory_order_acquire);
+  if (st == 0) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    st = d.state.load(std::memory_order_relaxed);
+    if (st == 0) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return AWQ_ERR_CUDA;
+      d.num_sms = sms;
+      st = (major == 10 && minor == 0) ? 1 : 2;
+      d.state.store(st, std::memory_order_release);
+    }
+  }
+  if (st != 1) return AWQ_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  if (sms_out) *sms_out = d.num_sms;
+  return AWQ_OK;
+}
+
+inline awq_status_t launch_status() { return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename Kernel>
+awq_status_t ensure_smem(Kernel kernel, int bytes, int dev, std::atomic<uint64_t>& done_mask) {
+  const uint64_t bit = 1ull << dev;
+  if (done_mask.load(std::memory_order_acquire) & bit) return AWQ_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return AWQ_OK;
+}
+
+// --------------------------------------------------------------------------- TMA descriptor
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// x' [M, K] fp16 row-major, box {64 k, BT tokens}, 128-byte swizzle, zero fill out of bounds.
+awq_status_t make_x_map(CUtensorMap* map, const void* x, int M, int K, int BT) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return AWQ_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kKTile), static_cast<cuuint32_t>(BT)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+// --------------------------------------------------------------------------- cluster launch helper
+template <typename... KArgs, typename... Args>
+awq_status_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_y, size_t smem,
+                            cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(cluster_y);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return AWQ_ERR_CUDA;
+  }
+  return AWQ_OK;
+}
+
+// --------------------------------------------------------------------------- decode dispatch
+template <int MT, int NT, int RW, int D>
+awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
+                             int M, int N, int K, int num_sms, cudaStream_t stream) {
+  using Cfg = GemvCfg<MT, NT, RW, D>;
+  const int row_blocks = padded_rows(N) / Cfg::kRows;
+  const int G = K / kGroup;
+  // cluster K-split: enough CTAs for about two per SM, at most 8 (portable), at most one per group
+  int cl = 1;
+  while (cl < 8 && cl * 2 <= G && row_blocks * cl < 2 * num_sms) cl *= 2;
+  const size_t smem = static_cast<size_t>(Cfg::kRows) * M * sizeof(float);
+  return launch_cluster(gemv_kernel<MT, NT, RW, D>, dim3(row_blocks, cl, 1), dim3(Cfg::kThreads, 1, 1), cl, smem,
+                        stream, x, qw, sc, zr, y, M, N, K);
+}
+
+awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
+                         int N, int K, int num_sms, cudaStream_t stream) {
+  const int mt = (M + 7) / 8;
+  switch (mt) {
+    case 1: return launch_gemv_cfg<1, 2, 4, 8>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
+    case 2: return launch_gemv_cfg<2, 2, 4, 6>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
+    case 3: return launch_gemv_cfg<3, 2, 4, 4>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
+    default: return launch_gemv_cfg<4, 2, 4, 4>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
+  }
+}
+
+// --------------------------------------------------------------------------- prefill dispatch
+template <int BT, int STAGES, int NDQ>
+awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
+                             int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  using C = GemmCfg<BT, STAGES, NDQ>;
+  static std::atomic<uint64_t> smem_done{0};
+  awq_status_t st = ensure_smem(gemm_kernel<BT, STAGES, NDQ>, C::kSmem, dev, smem_done);
+  if (st != AWQ_OK) return st;
+  CUtensorMap map;
+  st = make_x_map(&map, x, M, K, BT);
+  if (st != AWQ_OK) return st;
+  const long long tiles = static_cast<long long>(padded_rows(N) / kSuperRows) * ((M + BT - 1) / BT);
+  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms));
+  gemm_kernel<BT, STAGES, NDQ><<<grid, C::kThreads, C::kSmem, stream>>>(map, qw, sc, zr, y, M, N, K);
+  return launch_status();
+}
+
+awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
+                         int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  const long long nst = padded_rows(N) / kSuperRows;
+  auto tiles = [&](int bt) { return nst * ((M + bt - 1) / bt); };
+  if (M > 128 && tiles(256) >= num_sms)
+    return launch_gemm_cfg<256, 4, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  if (M > 64 && tiles(128) >= (num_sms * 3) / 4)
+    return launch_gemm_cfg<128, 6, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  if (M > 32) return launch_gemm_cfg<64, 7, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  return launch_gemm_cfg<32, 8, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+}
+
+awq_status_t check_linear_args(const void* x, const void* qw, const void* sc, const void* zr, const void* y, int M,
+                               int N, int K) {
+  if (!x || !qw || !sc || !zr || !y) return AWQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < kGroup || K % kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (static_cast<long long>(M) * K > (1ll << 31) - 1 || static_cast<long long>(padded_rows(N)) * K > (1ll << 34))
+    return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(qw) || !aligned16(sc) || !aligned16(zr) || !aligned16(y)) return AWQ_ERR_MISALIGNED;
+  return AWQ_OK;
+}
+
+}  // namespace
+}  // namespace awq
+
+using namespace awq;
+
+extern "C" {
+
+int awq_layout_version(void) { return 1; }
+
+const char* awq_status_string(int status) {
+  switch (status) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG: null pointer or size out of range";
+    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: configuration or device not supported";
+    case AWQ_ERR_MISALIGNED: return "AWQ_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA runtime error";
+    case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    default: return "AWQ_ERR_UNKNOWN";
+  }
+}
+
+awq_status_t awq_check_config(int bits, int group_size, int zero_point) {
+  return (bits == 4 && group_size == kGroup && zero_point == 1) ? AWQ_OK : AWQ_ERR_UNSUPPORTED;
+}
+
+size_t awq_qweight_bytes(int N, int K) {
+  if (N < 1 || K < kGroup || K % kGroup) return 0;
+  return static_cast<size_t>(padded_rows(N)) * K / 2;
+}
+size_t awq_scales_bytes(int N, int K) {
+  if (N < 1 || K < kGroup || K % kGroup) return 0;
+  return static_cast<size_t>(padded_rows(N)) * (K / kGroup) * 2;
+}
+size_t awq_zeros_bytes(int N, int K) {
+  if (N < 1 || K < kGroup || K % kGroup) return 0;
+  return static_cast<size_t>(padded_rows(N)) * (K / kGroup) / 2;
+}
+
+awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha, float* s_out, uint16_t* x_scaled,
+                                  awq_stream_t stream) {
+  if (!x || !s_out) return AWQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || K % 8 != 0 || static_cast<long long>(M) * K > (1ll << 40)) return AWQ_ERR_INVALID_ARG;
+  if (!(alpha == alpha) || alpha > 3.0e38f || alpha < -3.0e38f) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_scaled) || (reinterpret_cast<uintptr_t>(s_out) & 3u)) return AWQ_ERR_MISALIGNED;
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  int cl = 1;
+  while (cl < 8 && cl * 256 < M) cl *= 2;
+  const int slabs = (K + kActCols - 1) / kActCols;
+  return launch_cluster(act_scale_kernel, dim3(slabs, cl, 1), dim3(kActThreads, 1, 1), cl, 0,
+                        reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), M, K, alpha,
+                        s_out, reinterpret_cast<__half*>(x_scaled));
+}
+
+awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int K, uint16_t* x_scaled,
+                                   awq_stream_t stream) {
+  if (!x || !s || !x_scaled) return AWQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 1 || K % 8 != 0 || static_cast<long long>(M) * K > (1ll << 40)) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(s) || !aligned16(x_scaled)) return AWQ_ERR_MISALIGNED;
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  const long long total8 = static_cast<long long>(M) * K / 8;
+  const long long blocks = (total8 + 255) / 256;
+  if (blocks > 2147483647ll) return AWQ_ERR_INVALID_ARG;
+  scale_activations_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __half*>(x), s, total8, K, reinterpret_cast<__half*>(x_scaled));
+  return launch_status();
+}
+
+awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K, uint32_t* qweight,
+                               uint16_t* scales, uint8_t* zeros, awq_stream_t stream) {
+  if (!W || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
+  if (N < 1 || K < kGroup || K % kGroup != 0) return AWQ_ERR_INVALID_ARG;
+  if (static_cast<long long>(padded_rows(N)) * K > (1ll << 34)) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(fold_scale))
+    return AWQ_ERR_MISALIGNED;
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  const dim3 grid(K / kGroup, padded_rows(N) / kSuperRows, 1);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fold_scale)
+    quantize_g128_kernel<true><<<grid, kQuantThreads, 0, s>>>(reinterpret_cast<const __half*>(W), fold_scale, N, K,
+                                                                qweight, reinterpret_cast<__half*>(scales), zeros);
+  else
+    quantize_g128_kernel<false><<<grid, kQuantThreads, 0, s>>>(reinterpret_cast<const __half*>(W), nullptr, N, K,
+                                                                 qweight, reinterpret_cast<__half*>(scales), zeros);
+  return launch_status();
+}
+
+awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                            uint16_t* y, int M, int N, int K, awq_stream_t stream) {
+  awq_status_t st = check_linear_args(x, qweight, scales, zeros, y, M, N, K);
+  if (st != AWQ_OK) return st;
+  if (M > 32) return AWQ_ERR_INVALID_ARG;
+  int dev, sms;
+  st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  return launch_gemv(reinterpret_cast<const __half*>(x), qweight, reinterpret_cast<const __half*>(scales), zeros,
+                     reinterpret_cast<__half*>(y), M, N, K, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                            uint16_t* y, int M, int N, int K, awq_stream_t stream) {
+  awq_status_t st = check_linear_args(x, qweight, scales, zeros, y, M, N, K);
+  if (st != AWQ_OK) return st;
+  int dev, sms;
+  st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  return launch_gemm(reinterpret_cast<const __half*>(x), qweight, reinterpret_cast<const __half*>(scales), zeros,
+                     reinterpret_cast<__half*>(y), M, N, K, dev, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
+                              uint16_t* y, int M, int N, int K, awq_stream_t stream) {
+  if (M >= 1 && M <= 32) return awq_w4a16_gemv(x, qweight, scales, zeros, y, M, N, K, stream);
+  return awq_w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream);
+}
+
+awq_status_t awq_poll_device_status(awq_stream_t stream) {
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return AWQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(int)) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (v == 0) return AWQ_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int)) != cudaSuccess) return AWQ_ERR_CUDA;
+  return (v & kDevStatusTimeout) ? AWQ_ERR_TIMEOUT : AWQ_ERR_CUDA;
+}
+
+awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns) {
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  const unsigned long long v = ns ? ns : kDefaultWaitBudgetNs;
+  if (cudaDeviceSynchronize() != cudaSuccess) return AWQ_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_wait_budget_ns, &v, sizeof(v)) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+}  // extern "C"
