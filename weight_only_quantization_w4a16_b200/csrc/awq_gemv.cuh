@@ -177,12 +177,11 @@ __global__ void __launch_bounds__(GemvCfg<MT, NT, RW, D>::kThreads) gemv_kernel(
             }
           }
         }
-        // refill: activations 2 k-tiles ahead, weights D k-tiles ahead
+        // refill: activations 2 k-tiles ahead, weights D k-tiles ahead; a group's scale and
+        // zero slot is refilled only after the group's second k-tile has used it
         if (kl + 2 < nkt) issue_x(kl + 2, xring[u & 1]);
-        if (kl + D < nkt) {
-          issue_w(kl + D, wring[u]);
-          if ((u & 1) == 0) issue_meta(kl + D, sring[u / 2], zring[u / 2]);
-        }
+        if (kl + D < nkt) issue_w(kl + D, wring[u]);
+        if ((u & 1) && kl + D - 1 < nkt) issue_meta(kl + D - 1, sring[u / 2], zring[u / 2]);
       }
     }
   }
