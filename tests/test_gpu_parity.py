@@ -33,7 +33,7 @@ def _cuda():
 
 
 # ----------------------------------------------------------------------------- a1
-@pytest.mark.parametrize("M,K", [(1, 512), (7, 384), (33, 4096), (300, 1280), (1000, 11008), (4096, 512)])
+@pytest.mark.parametrize("M,K", [(1, 512), (7, 384), (32, 2048), (33, 4096), (300, 1280), (1000, 11008), (4096, 512)])
 def test_activation_scale_bit_exact(M, K):
     P = lib()
     x, _ = workloads.random_case(11, M, 16, K)

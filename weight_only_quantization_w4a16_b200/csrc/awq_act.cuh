@@ -139,6 +139,30 @@ __global__ void __launch_bounds__(kActThreads) act_scale_kernel(const __half* __
   }
 }
 
+// Small M (decode): one thread per column, no cluster. The same exact integer column sum,
+// the same float64 statistic and the same fp32 division as act_scale_kernel.
+constexpr int kActSmallMaxM = 32;
+__global__ void __launch_bounds__(128) act_scale_small_kernel(const __half* __restrict__ x, int M, int K,
+                                                             float alpha, float* __restrict__ s_out,
+                                                             __half* __restrict__ x_scaled) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  const unsigned short* xb = reinterpret_cast<const unsigned short*>(x);
+  uint64_t tot = 0;
+  for (int m = 0; m < M; ++m) tot += f16_abs_units(__ldg(xb + static_cast<size_t>(m) * K + k));
+  const double sum = __dmul_rn(static_cast<double>(tot), 0x1p-24);
+  double mean = __ddiv_rn(sum, static_cast<double>(M));
+  mean = fmax(mean, 1e-8);
+  const double p = (alpha == 0.5f) ? __dsqrt_rn(mean) : pow(mean, static_cast<double>(alpha));
+  const float sf = __double2float_rn(p);
+  s_out[k] = sf;
+  if (x_scaled == nullptr) return;
+  for (int m = 0; m < M; ++m) {
+    const size_t off = static_cast<size_t>(m) * K + k;
+    x_scaled[off] = __float2half_rn(__fdiv_rn(__half2float(__ushort_as_half(__ldg(xb + off))), sf));
+  }
+}
+
 // x'[m, k] = fp16_rn(fp32(x[m, k]) / s[k]) with a given s (the activation half of the
 // equivalent transform at inference time, s fixed by calibration). One thread per 8 values.
 __global__ void __launch_bounds__(256) scale_activations_kernel(const __half* __restrict__ x,

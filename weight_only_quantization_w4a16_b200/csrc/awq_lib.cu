@@ -130,28 +130,104 @@ awq_status_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, int
 }
 
 // --------------------------------------------------------------------------- decode dispatch
-template <int MT, int NT, int RW, int D>
-awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
-                             int M, int N, int K, int num_sms, cudaStream_t stream) {
-  using Cfg = GemvCfg<MT, NT, RW, D>;
-  const int row_blocks = padded_rows(N) / Cfg::kRows;
-  const int G = K / kGroup;
-  // cluster K-split: enough CTAs for about two per SM, at most 8 (portable), at most one per group
-  int cl = 1;
-  while (cl < 8 && cl * 2 <= G && row_blocks * cl < 2 * num_sms) cl *= 2;
-  const size_t smem = static_cast<size_t>(Cfg::kRows) * M * sizeof(float);
-  return launch_cluster(gemv_kernel<MT, NT, RW, D>, dim3(row_blocks, cl, 1), dim3(Cfg::kThreads, 1, 1), cl, smem,
-                        stream, x, qw, sc, zr, y, M, N, K);
+// Max co-resident clusters of a kernel for a cluster size and a dynamic shared-memory size;
+// cached (per kernel instantiation) because the occupancy query costs host time.
+struct ClusterOccCache {
+  std::mutex mu;
+  struct Entry { int dev, cl; size_t smem; int clusters; };
+  Entry e[256];
+  int n = 0;
+};
+template <typename Kernel>
+int max_active_clusters(Kernel kernel, int threads, size_t smem, int cl, int dev, ClusterOccCache& cache) {
+  {
+    std::lock_guard<std::mutex> lock(cache.mu);
+    for (int i = 0; i < cache.n; ++i)
+      if (cache.e[i].dev == dev && cache.e[i].cl == cl && cache.e[i].smem == smem) return cache.e[i].clusters;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cl, cl, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(cl);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lock(cache.mu);
+  if (cache.n < 256) cache.e[cache.n++] = {dev, cl, smem, n};
+  return n;
 }
 
+template <int MT, int S, int KS>
+awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
+                             int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  using Cfg = GemvCfg<MT, S, KS>;
+  auto kernel = gemv_kernel<MT, S, KS>;
+  constexpr int kMaxSmem = 227 * 1024;
+  static std::atomic<uint64_t> smem_done{0};
+  awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
+  if (st != AWQ_OK) return st;
+  CUtensorMap map;
+  st = make_x_map(&map, x, M, K, Cfg::kMP);
+  if (st != AWQ_OK) return st;
+  const int NST = padded_rows(N) / kSuperRows;
+  const int G = K / kGroup;
+  static ClusterOccCache cache;
+  // For each cluster size (K-split), find the co-resident cluster count C whose per-CTA partial
+  // buffers (ceil(NST / C) super-tiles) still let C clusters fit; cost = rounds x K-slice + a
+  // constant for the final reduction. The stream never synchronises before the end.
+  int best_cl = 0, best_clusters = 0, best_units = 0;
+  double best_cost = 1e300;
+  for (int cl = 1; cl <= 8; cl *= 2) {
+    if (cl > G) break;
+#ifdef AWQ_GEMV_FORCE_CL
+    if (cl != AWQ_GEMV_FORCE_CL) continue;
+#endif
+    int clusters = max_active_clusters(kernel, Cfg::kThreads, Cfg::smem_bytes(M, 1), cl, dev, cache);
+    int units = 0;
+    for (int it = 0; it < 6 && clusters > 0; ++it) {
+      clusters = std::min(clusters, NST);
+      units = (NST + clusters - 1) / clusters;
+      const size_t smem = Cfg::smem_bytes(M, units);
+      if (smem > static_cast<size_t>(kMaxSmem)) { clusters = 0; break; }
+      const int c2 = max_active_clusters(kernel, Cfg::kThreads, smem, cl, dev, cache);
+      if (c2 >= clusters) break;
+      clusters = c2;
+    }
+    if (clusters <= 0) continue;
+    const double cost = units * static_cast<double>((G + cl - 1) / cl) + 4.0;
+    if (cost < best_cost) { best_cost = cost; best_cl = cl; best_clusters = clusters; best_units = units; }
+  }
+  if (best_cl == 0) return AWQ_ERR_UNSUPPORTED;
+  return launch_cluster(kernel, dim3(best_clusters, best_cl, 1), dim3(Cfg::kThreads, 1, 1), best_cl,
+                        Cfg::smem_bytes(M, best_units), stream, map, qw, sc, zr, y, M, N, K, best_units);
+}
+
+// Compile-time tuning of the decode kernel for M <= 8 (stages, k-tiles per stage).
+#ifndef AWQ_GEMV1_STAGES
+#define AWQ_GEMV1_STAGES 4
+#endif
+#ifndef AWQ_GEMV1_KS
+#define AWQ_GEMV1_KS 4
+#endif
+
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
-                         int N, int K, int num_sms, cudaStream_t stream) {
+                         int N, int K, int dev, int num_sms, cudaStream_t stream) {
   const int mt = (M + 7) / 8;
   switch (mt) {
-    case 1: return launch_gemv_cfg<1, 2, 4, 8>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
-    case 2: return launch_gemv_cfg<2, 2, 4, 6>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
-    case 3: return launch_gemv_cfg<3, 2, 4, 4>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
-    default: return launch_gemv_cfg<4, 2, 4, 4>(x, qw, sc, zr, y, M, N, K, num_sms, stream);
+    case 1:
+      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 2: return launch_gemv_cfg<2, 3, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 3: return launch_gemv_cfg<3, 3, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default: return launch_gemv_cfg<4, 4, 2>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   }
 }
 
@@ -241,6 +317,11 @@ awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha, 
   int dev, sms;
   awq_status_t st = current_device(&dev, &sms);
   if (st != AWQ_OK) return st;
+  if (M <= kActSmallMaxM) {
+    act_scale_small_kernel<<<(K + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const __half*>(x), M, K, alpha, s_out, reinterpret_cast<__half*>(x_scaled));
+    return launch_status();
+  }
   int cl = 1;
   while (cl < 8 && cl * 256 < M) cl *= 2;
   const int slabs = (K + kActCols - 1) / kActCols;
@@ -275,14 +356,33 @@ awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N
   int dev, sms;
   awq_status_t st = current_device(&dev, &sms);
   if (st != AWQ_OK) return st;
-  const dim3 grid(K / kGroup, padded_rows(N) / kSuperRows, 1);
+  // W [N, K] fp16 as a 2-D tensor: boxes of 64 k x 128 rows, 128-byte swizzle, rows >= N read as 0
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return AWQ_ERR_CUDA;
+  CUtensorMap map;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kSuperRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(W), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  static std::atomic<uint64_t> done_f{0}, done_n{0};
+  st = fold_scale ? ensure_smem(quantize_g128_kernel<true>, kQSmem, dev, done_f)
+                  : ensure_smem(quantize_g128_kernel<false>, kQSmem, dev, done_n);
+  if (st != AWQ_OK) return st;
+  const long long units = static_cast<long long>(padded_rows(N) / kSuperRows) * (K / kGroup);
+  const int grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(AWQ_QUANT_MINBLOCKS) * sms));
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (fold_scale)
-    quantize_g128_kernel<true><<<grid, kQuantThreads, 0, s>>>(reinterpret_cast<const __half*>(W), fold_scale, N, K,
-                                                                qweight, reinterpret_cast<__half*>(scales), zeros);
+    quantize_g128_kernel<true><<<grid, kQThreads, kQSmem, s>>>(map, fold_scale, N, K, qweight,
+                                                                reinterpret_cast<__half*>(scales), zeros);
   else
-    quantize_g128_kernel<false><<<grid, kQuantThreads, 0, s>>>(reinterpret_cast<const __half*>(W), nullptr, N, K,
-                                                                 qweight, reinterpret_cast<__half*>(scales), zeros);
+    quantize_g128_kernel<false><<<grid, kQThreads, kQSmem, s>>>(map, nullptr, N, K, qweight,
+                                                                 reinterpret_cast<__half*>(scales), zeros);
   return launch_status();
 }
 
@@ -295,7 +395,7 @@ awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const ui
   st = current_device(&dev, &sms);
   if (st != AWQ_OK) return st;
   return launch_gemv(reinterpret_cast<const __half*>(x), qweight, reinterpret_cast<const __half*>(scales), zeros,
-                     reinterpret_cast<__half*>(y), M, N, K, sms, reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<__half*>(y), M, N, K, dev, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,

@@ -12,19 +12,25 @@
 //   q   = clamp(rint(w' / S) + z, 0, 15)
 //
 // w'/S is computed as va = w'*r, rho = fma(-S, va, w'), v = fma(rho, r, va)
-// with r = RN(1/S). This equals the IEEE quotient RN(w'/S) for every fp16
+// with r = RN(1/S), on packed fp32 pairs. This equals the IEEE quotient RN(w'/S) for every fp16
 // pair: w' and S carry at most 11 significant bits, so their exact quotient
 // is never a rounding midpoint of fp32 and lies at least 2^-12 ulp away from
 // one, while va is within 1.5 ulp of the quotient, rho is exact (at most 12
 // significant bits), and va + rho*r is within 2^-23 ulp of the quotient.
 // (S = inf gives NaN here and 0 in the IEEE quotient; both end as code 0
-// because z = 0 whenever S = inf.)
+// because z = 0 whenever S = inf.) Rounding and clamping use
+// clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z; the rint is
+// a magic-constant addition whose low byte feeds the byte-permute packing
+// directly (a clamped NaN becomes -z, i.e. code 0, as in the IEEE form).
 //
-// Work decomposition: a CTA of 8 warps owns one 128-row super-tile and one
-// group; warp nt owns rows nt*16 .. nt*16+15. Lane l loads row l/2, 16-byte
-// chunks c = 2i + (l&1) of the group (two lanes read one 32-byte sector per
-// instruction). Rows r and r+8 live in lanes l and l^16, which trade 4-code
-// quads with one shuffle per word to assemble packed layout v1.
+// Work decomposition: persistent CTAs walk (super-tile, group) units. A
+// producer lane streams each unit (128 rows x 128 k of fp16 W as two 2-D TMA
+// boxes with 128-byte swizzle, plus the group's fold scales) into a 3-stage
+// shared-memory ring, so HBM reads stay in flight while the 8 compute warps
+// (16 rows each) work. Lanes l and l^8 hold the two halves of one row's group
+// (their swizzled 16-byte reads are bank-conflict free); rows r and r+8 live
+// in lanes l and l^16, which trade 4-code quads with one shuffle per word to
+// assemble packed layout v1.
 #pragma once
 
 #include "awq_common.cuh"
@@ -33,125 +39,245 @@ namespace awq {
 
 constexpr int kQuantThreads = 256;
 
-__device__ __forceinline__ uint32_t quad_of_codes(float q0, float q1, float q2, float q3) {
-  // codes are integer-valued floats in [0, 15]; byte e = code of slot e
-  const uint32_t a = static_cast<uint32_t>(__float2int_rz(q0)) | (static_cast<uint32_t>(__float2int_rz(q1)) << 8);
-  const uint32_t b = static_cast<uint32_t>(__float2int_rz(q2)) | (static_cast<uint32_t>(__float2int_rz(q3)) << 8);
-  return a | (b << 16);
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two IEEE
+// fp32 operations, each rounded to nearest even exactly as the scalar form.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
+// Rounding by magic addition: for |v| <= 16, v + (1.5*2^23 + 16) rounds v to the
+// nearest integer n (ties to even, since the constant is even) and leaves 16 + n in the
+// low byte of the float's bits.
+constexpr float kRoundMagic = 12582928.0f;   // 1.5 * 2^23 + 16
+
+// One (super-tile, group) unit: 128 rows x 128 k of W, two 64-k TMA boxes with 128-byte
+// swizzle (16 KB each), plus the group's 128 fold scales.
+#ifndef AWQ_QUANT_STAGES
+#define AWQ_QUANT_STAGES 3
+#endif
+#ifndef AWQ_QUANT_MINBLOCKS
+#define AWQ_QUANT_MINBLOCKS 2
+#endif
+constexpr int kQStages = AWQ_QUANT_STAGES;
+constexpr int kQBox = kSuperRows * 64 * 2;                  // 16 KB
+// stage bases must stay 1024-byte aligned: the 128-byte swizzle pattern is a function of the address
+constexpr int kQStageBytes = (2 * kQBox + kGroup * 4 + 1023) / 1024 * 1024;   // 32 KB + 512 B, rounded up
+constexpr int kQComputeWarps = 8;
+constexpr int kQThreads = (kQComputeWarps + 1) * 32;        // + 1 producer warp
+constexpr int kQSmem = kQStages * kQStageBytes + 2 * kQStages * 8 + 16 + 1024;
+
 template <bool kFold>
-__global__ void __launch_bounds__(kQuantThreads) quantize_g128_kernel(const __half* __restrict__ W,
-                                                                     const float* __restrict__ fold, int N, int K,
-                                                                     uint32_t* __restrict__ qweight,
-                                                                     __half* __restrict__ scales,
-                                                                     uint8_t* __restrict__ zeros) {
-  __shared__ __align__(16) float s_fold[kGroup];
-  const int g = blockIdx.x;
-  const int st = blockIdx.y;
+__global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                                                                 const float* __restrict__ fold, int N, int K,
+                                                                 uint32_t* __restrict__ qweight,
+                                                                 __half* __restrict__ scales,
+                                                                 uint8_t* __restrict__ zeros) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQStages * kQStageBytes);
+  uint64_t* empty = full + kQStages;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + kQStages);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = warp;
   const int G = K / kGroup;
   const int KT = K / kKTile;
-  if (kFold) {
-    if (threadIdx.x < kGroup / 4)
-      reinterpret_cast<float4*>(s_fold)[threadIdx.x] =
-          __ldg(reinterpret_cast<const float4*>(fold + static_cast<size_t>(g) * kGroup) + threadIdx.x);
-    __syncthreads();
+  const int ST = padded_rows(N) / kSuperRows;
+  const int units = ST * G;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQComputeWarps);
+    }
+    *s_abort = 0;
+    mbar_fence_init();
   }
-  const int rr = lane >> 1;              // row in the 16-row tile
-  const int half = lane & 1;
-  const int h = rr >> 3;                 // 0: rows 0-7 (lanes 0-15), 1: rows 8-15
-  const int r = rr & 7;
-  const int n = st * kSuperRows + nt * kTileRows + rr;
-  const bool valid = n < N;
+  __syncthreads();
+  const unsigned long long budget = g_wait_budget_ns;
 
-  // ---- load 64 weights: chunks c = 2i + half, k = 128g + 8c .. 8c+7
-  uint4 raw[8];
-  const __half* wrow = W + static_cast<size_t>(valid ? n : 0) * K + static_cast<size_t>(g) * kGroup;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    raw[i] = valid ? ldg_stream_v4(wrow + 8 * (2 * i + half)) : make_uint4(0, 0, 0, 0);
+  if (warp == kQComputeWarps) {
+    // ---------------------------------------------------------------- producer
+    if (lane != 0) return;
+    tma_prefetch_desc(&tmap_w);
+    int stage = 0;
+    uint32_t phase = 0, issued_mask = 0, last_par = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const int st = u / G, g = u % G;
+      if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) break;
+      uint8_t* dst = smem + stage * kQStageBytes;
+      mbar_arrive_expect_tx(&full[stage], 2 * kQBox + (kFold ? kGroup * 4 : 0));
+      tma_load_2d(dst, &tmap_w, g * kGroup, st * kSuperRows, &full[stage]);
+      tma_load_2d(dst + kQBox, &tmap_w, g * kGroup + 64, st * kSuperRows, &full[stage]);
+      if (kFold) bulk_g2s(dst + 2 * kQBox, fold + static_cast<size_t>(g) * kGroup, kGroup * 4, &full[stage]);
+      issued_mask |= 1u << stage;
+      last_par = (last_par & ~(1u << stage)) | (phase << stage);
+      if (++stage == kQStages) { stage = 0; phase ^= 1; }
+    }
+    int never = 0;
+    for (int s = 0; s < kQStages; ++s)
+      if (issued_mask & (1u << s)) mbar_wait_bounded(&full[s], (last_par >> s) & 1u, &never, kDrainBudgetNs);
+    return;
+  }
 
-  // ---- fold and min/max
-  __half2 mn = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));   // +inf
-  __half2 mx = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));   // -inf
-  uint32_t wq[8][4];
+  // ------------------------------------------------------------------ compute warps
+  // lanes l and l^8 share a row (two halves of the group); lanes l and l^16 hold rows r, r+8
+  const int nt = warp;
+  const int r = lane & 7;
+  const int half = (lane >> 3) & 1;
+  const int h = lane >> 4;
+  const int rr = r + 8 * h;                 // row in the 16-row tile
+  const int row_s = nt * kTileRows + rr;    // row in the super-tile (TMA box row)
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int st = u / G, g = u % G;
+    if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget)) break;
+    const uint8_t* sb = smem + stage * kQStageBytes;
+    // ---- 64 weights of this lane: chunks c = 2i + half (16 B each), box c>>3, unit c&7 ^ (row & 7)
+    uint4 raw[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t v[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    for (int i = 0; i < 8; ++i) {
+      const int c = 2 * i + half;
+      raw[i] = *reinterpret_cast<const uint4*>(sb + (c >> 3) * kQBox + row_s * 128 + (((c & 7) ^ (row_s & 7)) << 4));
+    }
+    float4 sv[8][2];
+    if (kFold) {
+      const float* sfold = reinterpret_cast<const float*>(sb + 2 * kQBox);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __half2 hv = *reinterpret_cast<const __half2*>(&v[j]);
-      if (kFold) {
-        const int kk = 8 * (2 * i + half) + 2 * j;
-        const float2 f = __half22float2(hv);
-        hv = __floats2half2_rn(__fmul_rn(f.x, s_fold[kk]), __fmul_rn(f.y, s_fold[kk + 1]));
+      for (int i = 0; i < 8; ++i) {
+        sv[i][0] = *reinterpret_cast<const float4*>(&sfold[8 * (2 * i + half)]);
+        sv[i][1] = *reinterpret_cast<const float4*>(&sfold[8 * (2 * i + half) + 4]);
       }
-      wq[i][j] = *reinterpret_cast<uint32_t*>(&hv);
-      mn = __hmin2(mn, hv);
-      mx = __hmax2(mx, hv);
     }
-  }
-  float lo = fminf(__low2float(mn), __high2float(mn));
-  float hi = fmaxf(__low2float(mx), __high2float(mx));
-  lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, 1));
-  hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, 1));
+    // the stage is in registers: hand it back to the producer
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (++stage == kQStages) { stage = 0; phase ^= 1; }
 
-  // ---- scale, zero point, reciprocal
-  const float range = fmaxf(__fsub_rn(hi, lo), 1e-5f);
-  const __half S = __float2half_rn(__fdiv_rn(range, 15.0f));
-  const float Sf = __half2float(S);
-  const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, Sf)), 0.0f), 15.0f);
-  const float rcp = __frcp_rn(Sf);
+    const int n = st * kSuperRows + row_s;
+    const bool valid = n < N;
 
-  // ---- codes: one quad (4 consecutive k = slots e0..e3) per (chunk i, step-half sb)
-  uint32_t quad[8][2];
+    // ---- fold (fp32 multiply, RNE to fp16) and min/max on half2
+    __half2 mn = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));   // +inf
+    __half2 mx = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));   // -inf
+    uint32_t wq[8][4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t v[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
-    for (int sb = 0; sb < 2; ++sb) {
-      float qf[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t pair = wq[i][2 * sb + (e >> 1)];
-        const unsigned short hb = static_cast<unsigned short>((e & 1) ? (pair >> 16) : (pair & 0xFFFFu));
-        const float w = __half2float(__ushort_as_half(hb));
-        const float va = __fmul_rn(w, rcp);
-        const float rho = __fmaf_rn(-Sf, va, w);
-        const float v = __fmaf_rn(rho, rcp, va);
-        qf[e] = fminf(fmaxf(__fadd_rn(rintf(v), zf), 0.0f), 15.0f);
+      for (int j = 0; j < 4; ++j) {
+        __half2 hv = *reinterpret_cast<const __half2*>(&v[j]);
+        if (kFold) {
+          const float2 f = __half22float2(hv);
+          const float4& a = sv[i][j >> 1];
+          const float s0 = (j & 1) ? a.z : a.x;
+          const float s1 = (j & 1) ? a.w : a.y;
+          const float2 p = f2_unpack(f2_mul(f2_pack(f.x, f.y), f2_pack(s0, s1)));
+          hv = __floats2half2_rn(p.x, p.y);
+        }
+        wq[i][j] = *reinterpret_cast<uint32_t*>(&hv);
+        mn = __hmin2(mn, hv);
+        mx = __hmax2(mx, hv);
       }
-      quad[i][sb] = valid ? quad_of_codes(qf[0], qf[1], qf[2], qf[3]) : 0u;
     }
-  }
+    float lo = fminf(__low2float(mn), __high2float(mn));
+    float hi = fmaxf(__low2float(mx), __high2float(mx));
+    lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, 8));
+    hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, 8));
 
-  // ---- assemble words: lane with h = 0 builds k-tile 2g, lane with h = 1 builds k-tile 2g+1.
-  // Chunk i covers k-tile (i >> 2), column block t = (i & 3), steps s = 2*half + sb.
-  uint32_t* out = qweight + (static_cast<size_t>(st) * KT + 2 * g + h) * kSuperChunkWords +
-                  static_cast<size_t>(nt) * kChunkWords;
+    // ---- scale, zero point, reciprocal
+    const float range = fmaxf(__fsub_rn(hi, lo), 1e-5f);
+    const __half S = __float2half_rn(__fdiv_rn(range, 15.0f));
+    const float Sf = __half2float(S);
+    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, Sf)), 0.0f), 15.0f);
+    const float rcp = __frcp_rn(Sf);
+    // clamp(rint(w/S) + z, 0, 15) == rint(w_c / S) + z with w clamped to [-z S, (15 - z) S]: the
+    // bounds, rounded to fp16, move w/S by at most 15 * 2^-11 < 1/2, so the rounded codes are the
+    // same; the clamp runs on fp16 pairs. A non-finite S (an overflowed fold) takes the fp32 path.
+    const bool finite_s = Sf < 3.0e38f;
+    const __half2 wlo = __float2half2_rn(-zf * Sf), whi = __float2half2_rn(__fsub_rn(15.0f, zf) * Sf);
+    const float vlo = -zf, vhi = __fsub_rn(15.0f, zf);
+    const uint64_t rcp2 = f2_pack(rcp, rcp), nS2 = f2_pack(-Sf, -Sf), magic2 = f2_pack(kRoundMagic, kRoundMagic);
+    const uint32_t zsub = (16u - static_cast<uint32_t>(__float2int_rz(zf))) * 0x01010101u;
+
+    // ---- codes: one quad (4 consecutive k = slots e0..e3) per (chunk i, step-half sb)
+    uint32_t quad[8][2];
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    uint32_t w2[2];
+    for (int i = 0; i < 8; ++i) {
 #pragma unroll
-    for (int sb = 0; sb < 2; ++sb) {
-      const uint32_t send = h ? quad[t][sb] : quad[4 + t][sb];
-      const uint32_t mine = h ? quad[4 + t][sb] : quad[t][sb];
-      const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-      const uint32_t a = h ? recv : mine;   // row r
-      const uint32_t b = h ? mine : recv;   // row r + 8
-      w2[sb] = __byte_perm(a | (b << 4), 0u, 0x3120);
+      for (int sbh = 0; sbh < 2; ++sbh) {
+        uint32_t lowbytes[2];
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+          __half2 hp = *reinterpret_cast<const __half2*>(&wq[i][2 * sbh + pr]);
+          if (finite_s) hp = __hmin2(__hmax2(hp, wlo), whi);
+          const float2 w = __half22float2(hp);
+          const uint64_t w2 = f2_pack(w.x, w.y);
+          // IEEE quotient w / S: va = w * r, rho = w - S * va (exact), v = va + rho * r
+          const uint64_t va = f2_mul(w2, rcp2);
+          const uint64_t rho = f2_fma(nS2, va, w2);
+          float2 v = f2_unpack(f2_fma(rho, rcp2, va));
+          if (!finite_s) {
+            v.x = fminf(fmaxf(v.x, vlo), vhi);
+            v.y = fminf(fmaxf(v.y, vlo), vhi);
+          }
+          const float2 tq = f2_unpack(f2_add(f2_pack(v.x, v.y), magic2));
+          lowbytes[pr] = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x0040);
+        }
+        // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, 15], no borrows
+        const uint32_t q4 = __byte_perm(lowbytes[0], lowbytes[1], 0x5410) - zsub;
+        quad[i][sbh] = valid ? q4 : 0u;
+      }
     }
-    *reinterpret_cast<uint2*>(out + (4 * r + t) * 4 + 2 * half) = make_uint2(w2[0], w2[1]);
-  }
 
-  // ---- scales and zero points
-  const size_t meta = (static_cast<size_t>(st) * G + g) * 8 + nt;
-  const int zi = valid ? __float2int_rz(zf) : 0;
-  const int z_hi = __shfl_xor_sync(0xFFFFFFFFu, zi, 16);
-  if (half == 0) {
-    scales[meta * 16 + 2 * r + h] = valid ? S : __ushort_as_half(0);
-    if (h == 0) zeros[meta * 8 + r] = static_cast<uint8_t>(zi | (z_hi << 4));
+    // ---- assemble words: lane with h = 0 builds k-tile 2g, lane with h = 1 builds k-tile 2g+1.
+    // Chunk i covers k-tile (i >> 2), column block t = (i & 3), steps s = 2*half + sbh.
+    uint32_t* out = qweight + (static_cast<size_t>(st) * KT + 2 * g + h) * kSuperChunkWords +
+                    static_cast<size_t>(nt) * kChunkWords;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      uint32_t w2[2];
+#pragma unroll
+      for (int sbh = 0; sbh < 2; ++sbh) {
+        const uint32_t send = h ? quad[t][sbh] : quad[4 + t][sbh];
+        const uint32_t mine = h ? quad[4 + t][sbh] : quad[t][sbh];
+        const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+        const uint32_t a = h ? recv : mine;   // row r
+        const uint32_t b = h ? mine : recv;   // row r + 8
+        w2[sbh] = __byte_perm(a | (b << 4), 0u, 0x3120);
+      }
+      *reinterpret_cast<uint2*>(out + (4 * r + t) * 4 + 2 * half) = make_uint2(w2[0], w2[1]);
+    }
+
+    // ---- scales and zero points
+    const size_t meta = (static_cast<size_t>(st) * G + g) * 8 + nt;
+    const int zi = valid ? __float2int_rz(zf) : 0;
+    const int z_hi = __shfl_xor_sync(0xFFFFFFFFu, zi, 16);
+    if (half == 0) {
+      scales[meta * 16 + 2 * r + h] = valid ? S : __ushort_as_half(0);
+      if (h == 0) zeros[meta * 8 + r] = static_cast<uint8_t>(zi | (z_hi << 4));
+    }
   }
 }
 
