@@ -196,17 +196,25 @@ def oracle_sample_step(layers_data, rows_per_layer):
 
 
 def cpu_baseline(layers_data, target_s=12.0, threads=1):
+    """The oracle, single-threaded, on about `target_s` seconds of the workload: the first rows of
+    every layer (all rows when that is not enough), repeated until the target is reached."""
     from threadpoolctl import threadpool_limits
+    max_rows = max(W.shape[0] for _, W in layers_data)
     with threadpool_limits(limits=threads):
         t = time.perf_counter()
-        w = oracle_sample_step(layers_data, 128)
+        oracle_sample_step(layers_data, 128)
         probe = time.perf_counter() - t
-        rows = int(max(128, min(8192, 128 * target_s / max(probe, 1e-3))))
+        rows = int(max(128, min(max_rows, 128 * target_s / max(probe, 1e-3))))
         t = time.perf_counter()
-        w = oracle_sample_step(layers_data, rows)
+        w, reps = 0, 0
+        while True:
+            w += oracle_sample_step(layers_data, rows)
+            reps += 1
+            if time.perf_counter() - t >= 0.8 * target_s or reps >= 20:
+                break
         dt = time.perf_counter() - t
     return {"value": 2.0 * w / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"oracle (NumPy, {threads} thread) on the first {rows} rows of every layer "
+            "sample": f"oracle (NumPy, {threads} thread) on the first {rows} rows of every layer, {reps} pass(es) "
                       f"(fold + quantize + dequantize + float64 matmul; activation statistic over all of x); "
                       f"{w} weights in {dt:.2f} s; value = fp16-equivalent weight bytes (2/weight) per second"}
 
@@ -313,18 +321,22 @@ def run_ours(args, world, rank, local):
     kernels = ["act_scale", "quantize", "gemv" if decode else "gemm"]
 
     def step(events=None):
-        for li, d in enumerate(L):
-            if events is not None:
-                events[li][0].record()
+        """One pass of the path over all layers, grouped by kernel: a1 for every layer, then a2,
+        then the linear layer (the layers are independent). `events` (4 per step) mark the groups."""
+        if events is not None:
+            events[0].record()
+        for d in L:
             P.awq_activation_scale(d["x"], 0.5, d["s"], d["xs"])
-            if events is not None:
-                events[li][1].record()
+        if events is not None:
+            events[1].record()
+        for d in L:
             P.awq_quantize_g128(d["W"], d["s"], d["packed"])
-            if events is not None:
-                events[li][2].record()
+        if events is not None:
+            events[2].record()
+        for d in L:
             lin(d["xs"], *d["packed"], d["N"], d["y"])
-            if events is not None:
-                events[li][3].record()
+        if events is not None:
+            events[3].record()
 
     stream = torch.cuda.Stream(device=dev)
     R = max(1, args.graph_steps)
@@ -370,8 +382,7 @@ def run_ours(args, world, rank, local):
         # per-kernel breakdown: the same R steps captured with external event-record nodes
         # between the kernels; the graph is replayed, and the last replay's R samples are read
         nb = R
-        ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in L]
-              for _ in range(nb)]
+        ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(nb)]
         g_ev = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_ev, stream=stream):
             for b in range(nb):
@@ -390,12 +401,11 @@ def run_ours(args, world, rank, local):
     ms_step = ms_total / steps
     weights_per_step = sum(d["N"] * d["K"] for d in L)
     value = weak_scaling_value(weights_per_step, steps, ms_total, world)
-    # per-kernel breakdown
+    # per-kernel breakdown: each kernel group (its launches for all layers) between two events
     per = {k: [] for k in kernels}
     for r in range(nb):
-        for li in range(len(L)):
-            for ki, k in enumerate(kernels):
-                per[k].append((li, ev[r][li][ki].elapsed_time(ev[r][li][ki + 1])))
+        for ki, k in enumerate(kernels):
+            per[k].append(ev[r][ki].elapsed_time(ev[r][ki + 1]))
     peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
@@ -403,28 +413,20 @@ def run_ours(args, world, rank, local):
     peak_src = "of measured" if peaks else "of fallback"
     breakdown = {}
     for k in kernels:
-        tot_ms = sum(t for _, t in per[k])
-        nl = len(per[k])
+        group_ms = float(np.mean(per[k]))           # all layers' launches of this kernel, one step
         if k == "act_scale":
-            work = sum(bytes_act_scale(M, L[li]["K"]) for li, _ in per[k])
+            work = sum(bytes_act_scale(M, d["K"]) for d in L)
         elif k == "quantize":
-            work = sum(bytes_quantize(L[li]["N"], L[li]["K"]) for li, _ in per[k])
+            work = sum(bytes_quantize(d["N"], d["K"]) for d in L)
         else:
-            work = sum(bytes_linear(M, L[li]["N"], L[li]["K"]) for li, _ in per[k])
-        gbs = work / (tot_ms * 1e-3) / 1e9
-        entry = {"launches_per_step": len(L), "avg_us": 1e3 * tot_ms / nl, "share_of_step": None,
+            work = sum(bytes_linear(M, d["N"], d["K"]) for d in L)
+        gbs = work / (group_ms * 1e-3) / 1e9
+        entry = {"launches_per_step": len(L), "avg_us": 1e3 * group_ms / len(L), "share_of_step": None,
                  "algorithmic_GBps": gbs, "frac_hbm": gbs / hbm_peak}
         if k in ("gemv", "gemm"):
-            eff = sum(2 * L[li]["N"] * L[li]["K"] for li, _ in per[k]) / (tot_ms * 1e-3) / 1e9
-            entry["effective_weight_GBps"] = eff
-            fl = sum(flops_linear(M, L[li]["N"], L[li]["K"]) for li, _ in per[k])
-            entry["TFLOPs"] = fl / (tot_ms * 1e-3) / 1e12
+            entry["effective_weight_GBps"] = sum(2 * d["N"] * d["K"] for d in L) / (group_ms * 1e-3) / 1e9
+            entry["TFLOPs"] = sum(flops_linear(M, d["N"], d["K"]) for d in L) / (group_ms * 1e-3) / 1e12
             entry["frac_tensor"] = entry["TFLOPs"] / tc_peak
-            entry["per_layer_us"] = {
-                wl.layers[li].name: 1e3 * float(np.mean([t for lj, t in per[k] if lj == li])) for li in range(len(L))}
-            entry["per_layer_effective_weight_GBps"] = {
-                wl.layers[li].name: 2 * L[li]["N"] * L[li]["K"] / (1e-3 * float(np.mean([t for lj, t in per[k] if lj == li]))) / 1e9
-                for li in range(len(L))}
         breakdown[k] = entry
     step_sum_us = sum(e["avg_us"] * e["launches_per_step"] for e in breakdown.values())
     for e in breakdown.values():
@@ -492,8 +494,9 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": bench_config(wl, M),
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(t_wall0, t_wall1), "breakdown": breakdown,
-        "breakdown_method": ("graph of %d steps with external CUDA event-record nodes between kernels, "
-                             "replayed %d times; samples from the last replay" % (nb, ev_reps)),
+        "breakdown_method": ("graph of %d steps, each with external CUDA event-record nodes around its "
+                             "a1 / a2 / linear kernel groups, replayed %d times; the last replay's samples "
+                             "are averaged" % (nb, ev_reps)),
         "ms_per_step_with_kernel_events": k0.elapsed_time(k1) / (ev_reps * nb),
         "timing": "CUDA events around %d replays of a captured graph of %d steps; inputs larger than L2" % (reps, R),
     }

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_enter();
   const uint32_t tmem_base = *s_tmem;
   const unsigned long long budget = g_wait_budget_ns;
 

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(GemvCfg<MT, S, KS>::kThreads, 1) gemv_kernel(
     mbar_fence_init();
   }
   __syncthreads();
+  pdl_enter();
   const unsigned long long budget = g_wait_budget_ns;
   bool ok = true;
   int stage = 0;

@@ -106,22 +106,32 @@ awq_status_t make_x_map(CUtensorMap* map, const void* x, int M, int K, int BT) {
   return r == CUDA_SUCCESS ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
-// --------------------------------------------------------------------------- cluster launch helper
+// --------------------------------------------------------------------------- launch helper
+// Every kernel is launched with programmatic stream serialization (PDL): it may start while the
+// previous kernel of the stream drains, runs its prologue, and waits (griddepcontrol.wait) before
+// touching global memory. cluster_y > 1 adds a (1, cluster_y, 1) thread-block cluster.
 template <typename... KArgs, typename... Args>
-awq_status_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_y, size_t smem,
-                            cudaStream_t stream, Args... args) {
+awq_status_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_y, size_t smem,
+                       cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(cluster_y);
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster_y > 0) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = static_cast<unsigned>(cluster_y);
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
     cudaGetLastError();
     return AWQ_ERR_CUDA;
@@ -207,8 +217,8 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
     if (cost < best_cost) { best_cost = cost; best_cl = cl; best_clusters = clusters; best_units = units; }
   }
   if (best_cl == 0) return AWQ_ERR_UNSUPPORTED;
-  return launch_cluster(kernel, dim3(best_clusters, best_cl, 1), dim3(Cfg::kThreads, 1, 1), best_cl,
-                        Cfg::smem_bytes(M, best_units), stream, map, qw, sc, zr, y, M, N, K, best_units);
+  return launch_ex(kernel, dim3(best_clusters, best_cl, 1), dim3(Cfg::kThreads, 1, 1), best_cl,
+                   Cfg::smem_bytes(M, best_units), stream, map, qw, sc, zr, y, M, N, K, best_units);
 }
 
 // Compile-time tuning of the decode kernel for M <= 8 (stages, k-tiles per stage).
@@ -244,8 +254,8 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
   if (st != AWQ_OK) return st;
   const long long tiles = static_cast<long long>(padded_rows(N) / kSuperRows) * ((M + BT - 1) / BT);
   const int grid = static_cast<int>(std::min<long long>(tiles, num_sms));
-  gemm_kernel<BT, STAGES, NDQ><<<grid, C::kThreads, C::kSmem, stream>>>(map, qw, sc, zr, y, M, N, K);
-  return launch_status();
+  return launch_ex(gemm_kernel<BT, STAGES, NDQ>, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), 0, C::kSmem, stream, map,
+                   qw, sc, zr, y, M, N, K);
 }
 
 awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
@@ -317,15 +327,14 @@ awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha, 
   int dev, sms;
   awq_status_t st = current_device(&dev, &sms);
   if (st != AWQ_OK) return st;
-  if (M <= kActSmallMaxM) {
-    act_scale_small_kernel<<<(K + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const __half*>(x), M, K, alpha, s_out, reinterpret_cast<__half*>(x_scaled));
-    return launch_status();
-  }
+  if (M <= kActSmallMaxM)
+    return launch_ex(act_scale_small_kernel, dim3((K + 127) / 128, 1, 1), dim3(128, 1, 1), 0, 0,
+                     reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), M, K, alpha, s_out,
+                     reinterpret_cast<__half*>(x_scaled));
   int cl = 1;
   while (cl < 8 && cl * 256 < M) cl *= 2;
   const int slabs = (K + kActCols - 1) / kActCols;
-  return launch_cluster(act_scale_kernel, dim3(slabs, cl, 1), dim3(kActThreads, 1, 1), cl, 0,
+  return launch_ex(act_scale_kernel, dim3(slabs, cl, 1), dim3(kActThreads, 1, 1), cl, 0,
                         reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), M, K, alpha,
                         s_out, reinterpret_cast<__half*>(x_scaled));
 }
@@ -341,9 +350,9 @@ awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int
   const long long total8 = static_cast<long long>(M) * K / 8;
   const long long blocks = (total8 + 255) / 256;
   if (blocks > 2147483647ll) return AWQ_ERR_INVALID_ARG;
-  scale_activations_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const __half*>(x), s, total8, K, reinterpret_cast<__half*>(x_scaled));
-  return launch_status();
+  return launch_ex(scale_activations_kernel, dim3(static_cast<unsigned>(blocks), 1, 1), dim3(256, 1, 1), 0, 0,
+                   reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), s, total8, K,
+                   reinterpret_cast<__half*>(x_scaled));
 }
 
 awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K, uint32_t* qweight,
@@ -378,12 +387,10 @@ awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N
   const int grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(AWQ_QUANT_MINBLOCKS) * sms));
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (fold_scale)
-    quantize_g128_kernel<true><<<grid, kQThreads, kQSmem, s>>>(map, fold_scale, N, K, qweight,
-                                                                reinterpret_cast<__half*>(scales), zeros);
-  else
-    quantize_g128_kernel<false><<<grid, kQThreads, kQSmem, s>>>(map, nullptr, N, K, qweight,
-                                                                 reinterpret_cast<__half*>(scales), zeros);
-  return launch_status();
+    return launch_ex(quantize_g128_kernel<true>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), 0, kQSmem, s, map,
+                     fold_scale, N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
+  return launch_ex(quantize_g128_kernel<false>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), 0, kQSmem, s, map,
+                   static_cast<const float*>(nullptr), N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
 }
 
 awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
