@@ -163,7 +163,11 @@ __global__ void __launch_bounds__(GemvCfg<MT, S, KS>::kThreads, 1) gemv_kernel(
             // nibbles 16q * 2^-24); an extra mma against an all-ones A fragment gives sum_k x'_mk
             // for the zero-point term: sum x (q - z) S = S (sum x q) - S z (sum x).
             // NACC independent accumulator chains per tile shorten the dependent-mma chains
+#ifdef AWQ_GEMV_NACC
+            constexpr int NACC = MT == 1 ? AWQ_GEMV_NACC : 1;
+#else
             constexpr int NACC = MT == 1 ? 4 : (MT == 2 ? 2 : 1);
+#endif
             float tq[NACC][2][MT][4], tx[NACC][MT][4];
 #pragma unroll
             for (int a = 0; a < NACC; ++a)

@@ -258,16 +258,21 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
                    qw, sc, zr, y, M, N, K);
 }
 
+// Compile-time tuning of the prefill kernel: dequantization warps.
+#ifndef AWQ_GEMM_NDQ
+#define AWQ_GEMM_NDQ 8
+#endif
+
 awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
   const long long nst = padded_rows(N) / kSuperRows;
   auto tiles = [&](int bt) { return nst * ((M + bt - 1) / bt); };
   if (M > 128 && tiles(256) >= num_sms)
-    return launch_gemm_cfg<256, 4, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    return launch_gemm_cfg<256, 4, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   if (M > 64 && tiles(128) >= (num_sms * 3) / 4)
-    return launch_gemm_cfg<128, 6, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  if (M > 32) return launch_gemm_cfg<64, 7, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  return launch_gemm_cfg<32, 8, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    return launch_gemm_cfg<128, 6, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  if (M > 32) return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
 }
 
 awq_status_t check_linear_args(const void* x, const void* qw, const void* sc, const void* zr, const void* y, int M,

@@ -22,6 +22,9 @@
 // clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z; the rint is
 // a magic-constant addition whose low byte feeds the byte-permute packing
 // directly (a clamped NaN becomes -z, i.e. code 0, as in the IEEE form).
+// Measured alternatives that were slower on B200 and are not used: clamping
+// w' on fp16 pairs before the division, a tree of min/max chains, and scalar
+// fp32 in place of the packed f32x2 pairs.
 //
 // Work decomposition: persistent CTAs walk (super-tile, group) units. A
 // producer lane streams each unit (128 rows x 128 k of fp16 W as two 2-D TMA
@@ -179,13 +182,9 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
     const int n = st * kSuperRows + row_s;
     const bool valid = n < N;
 
-    // ---- fold (fp32 multiply, RNE to fp16) and min/max on half2 (four independent chains)
-    __half2 mn[4], mx[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      mn[c] = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));   // +inf
-      mx[c] = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));   // -inf
-    }
+    // ---- fold (fp32 multiply, RNE to fp16) and min/max on half2
+    __half2 mn = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));   // +inf
+    __half2 mx = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));   // -inf
     uint32_t wq[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -198,22 +197,16 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
           const float4& a = sv[i][j >> 1];
           const float s0 = (j & 1) ? a.z : a.x;
           const float s1 = (j & 1) ? a.w : a.y;
-#ifdef AWQ_QUANT_SCALAR
-          hv = __floats2half2_rn(__fmul_rn(f.x, s0), __fmul_rn(f.y, s1));
-#else
           const float2 p = f2_unpack(f2_mul(f2_pack(f.x, f.y), f2_pack(s0, s1)));
           hv = __floats2half2_rn(p.x, p.y);
-#endif
         }
         wq[i][j] = *reinterpret_cast<uint32_t*>(&hv);
-        mn[j] = __hmin2(mn[j], hv);
-        mx[j] = __hmax2(mx[j], hv);
+        mn = __hmin2(mn, hv);
+        mx = __hmax2(mx, hv);
       }
     }
-    mn[0] = __hmin2(__hmin2(mn[0], mn[1]), __hmin2(mn[2], mn[3]));
-    mx[0] = __hmax2(__hmax2(mx[0], mx[1]), __hmax2(mx[2], mx[3]));
-    float lo = fminf(__low2float(mn[0]), __high2float(mn[0]));
-    float hi = fmaxf(__low2float(mx[0]), __high2float(mx[0]));
+    float lo = fminf(__low2float(mn), __high2float(mn));
+    float hi = fmaxf(__low2float(mx), __high2float(mx));
     lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, 8));
     hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, 8));
 
@@ -223,11 +216,7 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
     const float Sf = __half2float(S);
     const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, Sf)), 0.0f), 15.0f);
     const float rcp = __frcp_rn(Sf);
-    // clamp(rint(w/S) + z, 0, 15) == rint(w_c / S) + z with w clamped to [-z S, (15 - z) S]: the
-    // bounds, rounded to fp16, move w/S by at most 15 * 2^-11 < 1/2, so the rounded codes are the
-    // same; the clamp runs on fp16 pairs. A non-finite S (an overflowed fold) takes the fp32 path.
-    const bool finite_s = Sf < 3.0e38f;
-    const __half2 wlo = __float2half2_rn(-zf * Sf), whi = __float2half2_rn(__fsub_rn(15.0f, zf) * Sf);
+    // clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z, as -z and 15 - z are integers
     const float vlo = -zf, vhi = __fsub_rn(15.0f, zf);
     const uint64_t rcp2 = f2_pack(rcp, rcp), nS2 = f2_pack(-Sf, -Sf), magic2 = f2_pack(kRoundMagic, kRoundMagic);
     const uint32_t zsub = (16u - static_cast<uint32_t>(__float2int_rz(zf))) * 0x01010101u;
@@ -241,32 +230,15 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
         uint32_t lowbytes[2];
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr) {
-          __half2 hp = *reinterpret_cast<const __half2*>(&wq[i][2 * sbh + pr]);
-          if (finite_s) hp = __hmin2(__hmax2(hp, wlo), whi);
-          const float2 w = __half22float2(hp);
+          const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&wq[i][2 * sbh + pr]));
           // IEEE quotient w / S: va = w * r, rho = w - S * va (exact), v = va + rho * r
-#ifdef AWQ_QUANT_SCALAR
-          float2 v;
-          {
-            const float vax = __fmul_rn(w.x, rcp), vay = __fmul_rn(w.y, rcp);
-            v.x = __fmaf_rn(__fmaf_rn(-Sf, vax, w.x), rcp, vax);
-            v.y = __fmaf_rn(__fmaf_rn(-Sf, vay, w.y), rcp, vay);
-          }
-#else
           const uint64_t w2 = f2_pack(w.x, w.y);
           const uint64_t va = f2_mul(w2, rcp2);
           const uint64_t rho = f2_fma(nS2, va, w2);
           float2 v = f2_unpack(f2_fma(rho, rcp2, va));
-#endif
-          if (!finite_s) {
-            v.x = fminf(fmaxf(v.x, vlo), vhi);
-            v.y = fminf(fmaxf(v.y, vlo), vhi);
-          }
-#ifdef AWQ_QUANT_SCALAR
-          const float2 tq = make_float2(__fadd_rn(v.x, kRoundMagic), __fadd_rn(v.y, kRoundMagic));
-#else
+          v.x = fminf(fmaxf(v.x, vlo), vhi);
+          v.y = fminf(fmaxf(v.y, vlo), vhi);
           const float2 tq = f2_unpack(f2_add(f2_pack(v.x, v.y), magic2));
-#endif
           lowbytes[pr] = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x0040);
         }
         // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, 15], no borrows
