@@ -261,10 +261,10 @@ def metric_name(M):
 
 
 def bench_config(wl, M):
+    lin = "decode GEMV (a3)" if M <= 32 else "prefill GEMM (a4)"
     return {"workload": wl.name, "M": M,
             "layers": [{"name": l.name, "K": l.K, "N": l.N} for l in wl.layers],
-            "step": "per layer: activation statistic + scaling (a1), fold + 4-bit g128 quantizer (a2), "
-                    + ("decode GEMV (a3)" if M <= 32 else "prefill GEMM (a4)"),
+            "step": "per layer: activation statistic + scaling (a1), fold + 4-bit g128 quantizer (a2), " + lin,
             "weights": "int4, group 128 along K, fp16 scale, 4-bit zero point",
             "accumulate": "f32",
             "l2": "inputs larger than L2 (fp16 weights of the step: %.0f MB vs 126 MB L2)"
@@ -304,7 +304,6 @@ def run_ours(args, world, rank, local):
     wl = workloads.WORKLOADS[args.workload]
     M = args.m or wl.Ms[0]
     decode = M <= 32
-    lin = P.awq_w4a16_gemv if decode else P.awq_w4a16_gemm
 
     host = [workloads.layer_inputs(wl, i, M) for i in range(len(wl.layers))]
     L = []
@@ -317,6 +316,8 @@ def run_ours(args, world, rank, local):
              "y": torch.empty((M, N), dtype=torch.float16, device=dev)}
         d["packed"] = P.alloc_packed(N, K, dev)
         L.append(d)
+
+    lin = P.awq_w4a16_gemv if decode else P.awq_w4a16_gemm
 
     kernels = ["act_scale", "quantize", "gemv" if decode else "gemm"]
 
@@ -491,8 +492,8 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": metric_name(M), "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": warm_reps * R, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": bench_config(wl, M),
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": bench_config(wl, M), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks.summary(t_wall0, t_wall1), "breakdown": breakdown,
         "breakdown_method": ("graph of %d steps, each with external CUDA event-record nodes around its "
                              "a1 / a2 / linear kernel groups, replayed %d times; the last replay's samples "

@@ -173,6 +173,13 @@ AWQ_API awq_status_t awq_poll_device_status(awq_stream_t stream);
  * memory and returns. */
 AWQ_API awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns);
 
+/* Test hook: nonzero makes the producer of the quantizer and of the decode
+ * kernel skip the copies of its first pipeline stage, so the consumers' wait
+ * on that stage can only end by running out its budget (shorten it with
+ * awq_debug_set_wait_budget_ns). The kernel then behaves as described there.
+ * 0 restores normal operation. Synchronous; current device. */
+AWQ_API awq_status_t awq_debug_drop_first_copy(int enable);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

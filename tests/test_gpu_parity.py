@@ -244,3 +244,4 @@ def test_prefill_full_size_sampled(layer_idx, M):
                                             (1, 512, "awq_w4a16_gemm")])
 def test_70b_full_size_sampled(layer_idx, M, fn):
     _full_size_case("llama2_70b_layers", layer_idx, M, fn)
+

@@ -14,7 +14,8 @@ Functions (same names as the C ABI):
 * ``awq_w4a16_gemv(x, qweight, scales, zeros, N)`` -> y[M,N] fp16 (M <= 32)
 * ``awq_w4a16_gemm(x, qweight, scales, zeros, N)`` -> y[M,N] fp16
 * ``awq_w4a16_linear(...)``: gemv for M <= 32, gemm otherwise
-* ``awq_poll_device_status()``, ``awq_debug_set_wait_budget_ns(ns)``
+* ``awq_poll_device_status()``, test hooks ``awq_debug_set_wait_budget_ns(ns)``,
+  ``awq_debug_drop_first_copy(enable)``
 """
 from __future__ import annotations
 
@@ -63,6 +64,7 @@ _SIGS = {
     "awq_w4a16_linear": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_poll_device_status": ([_VP], _I),
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
+    "awq_debug_drop_first_copy": ([_I], _I),
 }
 
 
@@ -230,6 +232,10 @@ def awq_poll_device_status() -> int:
 
 def awq_debug_set_wait_budget_ns(ns: int) -> None:
     _check("awq_debug_set_wait_budget_ns", load_library().awq_debug_set_wait_budget_ns(int(ns)))
+
+
+def awq_debug_drop_first_copy(enable: bool) -> None:
+    _check("awq_debug_drop_first_copy", load_library().awq_debug_drop_first_copy(int(bool(enable))))
 
 
 class AWQLinear:

@@ -36,6 +36,9 @@ constexpr unsigned long long kDrainBudgetNs = 1000000000ull;         // 1 s for 
 // Defined here: the library is built as one translation unit (awq_lib.cu).
 __device__ int g_dev_status = 0;
 __device__ unsigned long long g_wait_budget_ns = kDefaultWaitBudgetNs;
+// Test hook: nonzero makes the producer of each pipelined kernel skip the copies of its first
+// ring stage, so the consumers' wait on that stage can only end by running out its budget.
+__device__ int g_debug_drop_first_copy = 0;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -86,15 +89,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with an explicit bound (ns) on how long the thread may stay suspended in it.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Budgets below this (set only through the test hook) also bound each suspended try_wait, so
+// that the budget is honoured even when the hardware's own suspend window is longer.
+constexpr unsigned long long kShortBudgetNs = 1000000ull;
+
 // Bounded wait: returns true when the phase with `parity` has completed.
 // Gives up (returns false) when *abort is set by another warp, or after
 // `budget_ns` of waiting, in which case it sets *abort and the device status.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   unsigned long long budget_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool short_budget = budget_ns < kShortBudgetNs;
+  const uint32_t hint = static_cast<uint32_t>(budget_ns);
+  auto try_once = [&]() { return short_budget ? mbar_try_wait_for(bar, parity, hint) : mbar_try_wait(bar, parity); };
+  if (try_once()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_once()) return true;
     if (*abort) return false;
     if (globaltimer_ns() - t0 > budget_ns) {
       *abort = 1;

@@ -61,8 +61,6 @@ awq_status_t current_device(int* dev_out, int* sms_out) {
   return AWQ_OK;
 }
 
-inline awq_status_t launch_status() { return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA; }
-
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
 template <typename Kernel>
 awq_status_t ensure_smem(Kernel kernel, int bytes, int dev, std::atomic<uint64_t>& done_mask) {
@@ -176,11 +174,11 @@ int max_active_clusters(Kernel kernel, int threads, size_t smem, int cl, int dev
   return n;
 }
 
-template <int MT, int S, int KS>
+template <int MT, int S, int KS, int CW>
 awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
                              int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using Cfg = GemvCfg<MT, S, KS>;
-  auto kernel = gemv_kernel<MT, S, KS>;
+  using Cfg = GemvCfg<MT, S, KS, CW>;
+  auto kernel = gemv_kernel<MT, S, KS, CW>;
   constexpr int kMaxSmem = 227 * 1024;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
@@ -229,15 +227,17 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
 #define AWQ_GEMV1_KS 4
 #endif
 
+// Consumer warps: 4 (two 16-row tiles each) up to M = 16; 8 (one tile each) above, where the
+// extra warps hide the longer mma chains (measured on the Llama-2-7B and 70B decode shapes).
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
   const int mt = (M + 7) / 8;
   switch (mt) {
     case 1:
-      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 2: return launch_gemv_cfg<2, 3, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 3: return launch_gemv_cfg<3, 3, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    default: return launch_gemv_cfg<4, 4, 2>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 2: return launch_gemv_cfg<2, 3, 4, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 3: return launch_gemv_cfg<3, 3, 4, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default: return launch_gemv_cfg<4, 4, 2, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   }
 }
 
@@ -438,6 +438,15 @@ awq_status_t awq_poll_device_status(awq_stream_t stream) {
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int)) != cudaSuccess) return AWQ_ERR_CUDA;
   return (v & kDevStatusTimeout) ? AWQ_ERR_TIMEOUT : AWQ_ERR_CUDA;
+}
+
+awq_status_t awq_debug_drop_first_copy(int enable) {
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  const int v = enable ? 1 : 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return AWQ_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_debug_drop_first_copy, &v, sizeof(v)) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
 awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns) {

@@ -117,7 +117,10 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
     mbar_fence_init();
   }
   __syncthreads();
-  pdl_enter();
+  // Wait for the previous kernel, but do not let the next one start early: kernels that read
+  // packed weights before their own wait (the split-K decode kernel) may follow, so the next
+  // kernel launches only once this grid has completed and every write below is visible.
+  pdl_wait();
   const unsigned long long budget = g_wait_budget_ns;
 
   if (warp == kQComputeWarps) {
@@ -126,9 +129,15 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
     tma_prefetch_desc(&tmap_w);
     int stage = 0;
     uint32_t phase = 0, issued_mask = 0, last_par = 0;
+    bool drop = g_debug_drop_first_copy != 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       const int st = u / G, g = u % G;
       if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) break;
+      if (drop) {   // test hook: this stage's copies are never issued
+        drop = false;
+        if (++stage == kQStages) { stage = 0; phase ^= 1; }
+        continue;
+      }
       uint8_t* dst = smem + stage * kQStageBytes;
       mbar_arrive_expect_tx(&full[stage], 2 * kQBox + (kFold ? kGroup * 4 : 0));
       tma_load_2d(dst, &tmap_w, g * kGroup, st * kSuperRows, &full[stage]);
@@ -275,6 +284,7 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
       if (h == 0) zeros[meta * 8 + r] = static_cast<uint8_t>(zi | (z_hi << 4));
     }
   }
+  __threadfence();   // this thread's codes, scales and zeros are visible device-wide before it exits
 }
 
 }  // namespace awq
