@@ -18,13 +18,16 @@
 // one, while va is within 1.5 ulp of the quotient, rho is exact (at most 12
 // significant bits), and va + rho*r is within 2^-23 ulp of the quotient.
 // (S = inf gives NaN here and 0 in the IEEE quotient; both end as code 0
-// because z = 0 whenever S = inf.) Rounding and clamping use
-// clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z; the rint is
-// a magic-constant addition whose low byte feeds the byte-permute packing
-// directly (a clamped NaN becomes -z, i.e. code 0, as in the IEEE form).
-// Measured alternatives that were slower on B200 and are not used: clamping
-// w' on fp16 pairs before the division, a tree of min/max chains, and scalar
-// fp32 in place of the packed f32x2 pairs.
+// because z = 0 whenever S = inf.) Rounding is a magic-constant addition
+// (1.5*2^23 + 16, even, so ties go to even). Clamping: when every lane's
+// group keeps |w'/S| inside a 16-bit window (all groups of finite weights
+// whose range is above the 1e-5 floor), the low 16 bits of the rounded sum
+// are clamped as packed integers by two DPX instructions; otherwise
+// clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z is taken in
+// fp32 before rounding (a clamped NaN becomes -z, i.e. code 0, as in the
+// IEEE form). Measured alternatives that were slower on B200 and are not
+// used: clamping w' on fp16 pairs before the division, a tree of min/max
+// chains, and scalar fp32 in place of the packed f32x2 pairs.
 //
 // Work decomposition: persistent CTAs walk (super-tile, group) units. A
 // producer lane streams each unit (128 rows x 128 k of fp16 W as two 2-D TMA
@@ -68,6 +71,18 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+// fp16 pair -> two fp32 values through the mixed-precision add f32(h) + (-0.0), exact for every
+// fp16 value (signed zeros and non-finite values included); measured slightly faster than the
+// conversion instruction here.
+__device__ __forceinline__ float2 h2_to_f2(uint32_t v) {
+  float a, b;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %3;\n\tadd.rn.f32.f16 %1, h, %3;\n\t}"
+      : "=f"(a), "=f"(b)
+      : "r"(v), "f"(-0.0f));
+  return make_float2(a, b);
 }
 
 // Rounding by magic addition: for |v| <= 16, v + (1.5*2^23 + 16) rounds v to the
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
       for (int j = 0; j < 4; ++j) {
         __half2 hv = *reinterpret_cast<const __half2*>(&v[j]);
         if (kFold) {
-          const float2 f = __half22float2(hv);
+          const float2 f = h2_to_f2(v[j]);
           const float4& a = sv[i][j >> 1];
           const float s0 = (j & 1) ? a.z : a.x;
           const float s1 = (j & 1) ? a.w : a.y;
@@ -232,27 +247,56 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
 
     // ---- codes: one quad (4 consecutive k = slots e0..e3) per (chunk i, step-half sb)
     uint32_t quad[8][2];
+    // Packed-integer clamp: for |v| < 2^15 - 16 the low 16 bits of v + (1.5*2^23 + 16) are
+    // 16 + rint(v) (two's complement); one DPX add-max-relu and one min-relu on 16-bit pairs then
+    // give clamp(rint(v) + z, 0, 15). Every group of finite fp16 weights whose range is not the
+    // 1e-5 floor has |v| <= 15 * 2^11 (range >= one fp16 ulp of max(|lo|, |hi|)); groups beyond
+    // the 16-bit window (range at the floor, non-finite values) take the fp32 clamp below.
+    const bool fast = fmaxf(fabsf(lo), fabsf(hi)) * rcp < 32000.0f;
+    if (__all_sync(0xFFFFFFFFu, fast)) {
+      const uint32_t zoff2 = (static_cast<uint32_t>(__float2int_rz(zf) - 16) & 0xFFFFu) * 0x00010001u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 8; ++i) {
 #pragma unroll
-      for (int sbh = 0; sbh < 2; ++sbh) {
-        uint32_t lowbytes[2];
+        for (int sbh = 0; sbh < 2; ++sbh) {
+          uint32_t code2[2];
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const float2 w = __half22float2(*reinterpret_cast<const __half2*>(&wq[i][2 * sbh + pr]));
-          // IEEE quotient w / S: va = w * r, rho = w - S * va (exact), v = va + rho * r
-          const uint64_t w2 = f2_pack(w.x, w.y);
-          const uint64_t va = f2_mul(w2, rcp2);
-          const uint64_t rho = f2_fma(nS2, va, w2);
-          float2 v = f2_unpack(f2_fma(rho, rcp2, va));
-          v.x = fminf(fmaxf(v.x, vlo), vhi);
-          v.y = fminf(fmaxf(v.y, vlo), vhi);
-          const float2 tq = f2_unpack(f2_add(f2_pack(v.x, v.y), magic2));
-          lowbytes[pr] = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x0040);
+          for (int pr = 0; pr < 2; ++pr) {
+            const float2 w = h2_to_f2(wq[i][2 * sbh + pr]);
+            const uint64_t w2 = f2_pack(w.x, w.y);
+            const uint64_t va = f2_mul(w2, rcp2);
+            const uint64_t rho = f2_fma(nS2, va, w2);
+            const uint64_t v2 = f2_fma(rho, rcp2, va);
+            const float2 tq = f2_unpack(f2_add(v2, magic2));
+            const uint32_t t16 = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x5410);
+            code2[pr] = __vimin_s16x2_relu(__viaddmax_s16x2_relu(t16, zoff2, 0u), 0x000F000Fu);
+          }
+          quad[i][sbh] = __byte_perm(code2[0], code2[1], 0x6420);
         }
-        // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, 15], no borrows
-        const uint32_t q4 = __byte_perm(lowbytes[0], lowbytes[1], 0x5410) - zsub;
-        quad[i][sbh] = valid ? q4 : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int sbh = 0; sbh < 2; ++sbh) {
+          uint32_t lowbytes[2];
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const float2 w = h2_to_f2(wq[i][2 * sbh + pr]);
+            // IEEE quotient w / S: va = w * r, rho = w - S * va (exact), v = va + rho * r
+            const uint64_t w2 = f2_pack(w.x, w.y);
+            const uint64_t va = f2_mul(w2, rcp2);
+            const uint64_t rho = f2_fma(nS2, va, w2);
+            float2 v = f2_unpack(f2_fma(rho, rcp2, va));
+            v.x = fminf(fmaxf(v.x, vlo), vhi);
+            v.y = fminf(fmaxf(v.y, vlo), vhi);
+            const float2 tq = f2_unpack(f2_add(f2_pack(v.x, v.y), magic2));
+            lowbytes[pr] = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x0040);
+          }
+          // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, 15], no borrows
+          const uint32_t q4 = __byte_perm(lowbytes[0], lowbytes[1], 0x5410) - zsub;
+          quad[i][sbh] = valid ? q4 : 0u;
+        }
       }
     }
 
