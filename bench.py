@@ -281,12 +281,15 @@ def kernel_source_hash(name):
         return None
 
 
-def profile_traffic(kernel_file):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+def profile_traffic(kernel_file, workload, M):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this workload and M
+    and the kernel source is unchanged since."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         d = json.load(open(p))
     except (OSError, ValueError):
+        return None
+    if d.get("_workload") != workload or d.get("_M") != M:
         return None
     e = d.get(kernel_file)
     if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
@@ -436,7 +439,7 @@ def run_ours(args, world, rank, local):
     dom = max(breakdown, key=lambda k: breakdown[k]["avg_us"] * breakdown[k]["launches_per_step"])
     kfile = {"act_scale": "awq_act.cuh", "quantize": "awq_quant.cuh", "gemv": "awq_gemv.cuh",
              "gemm": "awq_gemm.cuh"}[dom]
-    tr = profile_traffic(kfile)
+    tr = profile_traffic(kfile, wl.name, M)
     if dom == "gemm" and not decode:
         roof = {"bound": "tensor", "achieved": breakdown[dom]["TFLOPs"], "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": breakdown[dom]["TFLOPs"] / tc_peak, "traffic": tr["bytes_per_launch"] if tr else None,

@@ -140,12 +140,12 @@ __device__ __forceinline__ void gemv_group(float (&acc)[NT][MT][4], const uint8_
 }
 
 // MT: 8-token tiles (M <= 8*MT); S: pipeline stages; KS: 64-k tiles per stage (even);
-// CW: consumer warps (4 or 8). A CTA is one producer warp plus CW consumer warps; consumer
+// CW: consumer warps (2, 4 or 8). A CTA is one producer warp plus CW consumer warps; consumer
 // warp w owns rows (128/CW) w .. (128/CW)(w+1) - 1 of a 128-row super-tile (8/CW mma tiles).
 template <int MT, int S, int KS, int CW>
 struct GemvCfg {
   static_assert(KS % 2 == 0, "a stage must hold whole groups");
-  static_assert(CW == 4 || CW == 8, "4 or 8 consumer warps");
+  static_assert(CW == 2 || CW == 4 || CW == 8, "2, 4 or 8 consumer warps");
   static constexpr int kNT = 8 / CW;                         // 16-row tiles per consumer warp
   static constexpr int kMP = 8 * MT;                         // token rows of the activation boxes
   static constexpr int kX = KS * kMP * 128;                  // activations: KS boxes of 64 k x kMP rows

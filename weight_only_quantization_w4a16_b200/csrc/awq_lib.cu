@@ -219,25 +219,44 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
                    Cfg::smem_bytes(M, best_units), stream, map, qw, sc, zr, y, M, N, K, best_units);
 }
 
-// Compile-time tuning of the decode kernel for M <= 8 (stages, k-tiles per stage).
+// Compile-time tuning of the decode kernel per token tile: stages, 64-k tiles per stage,
+// consumer warps. Measured on the Llama-2-7B and 70B decode shapes: larger stages (fewer
+// barrier round trips per weight) win as long as two CTAs still fit on an SM; 4 consumer
+// warps up to M = 16, 8 above, where the extra warps hide the longer mma chains.
 #ifndef AWQ_GEMV1_STAGES
-#define AWQ_GEMV1_STAGES 4
+#define AWQ_GEMV1_STAGES 2
 #endif
 #ifndef AWQ_GEMV1_KS
-#define AWQ_GEMV1_KS 4
+#define AWQ_GEMV1_KS 8
+#endif
+#ifndef AWQ_GEMV1_CW
+#define AWQ_GEMV1_CW 4
+#endif
+#ifndef AWQ_GEMV2_STAGES
+#define AWQ_GEMV2_STAGES 3
+#endif
+#ifndef AWQ_GEMV2_KS
+#define AWQ_GEMV2_KS 4
+#endif
+#ifndef AWQ_GEMV4_STAGES
+#define AWQ_GEMV4_STAGES 3
+#endif
+#ifndef AWQ_GEMV4_KS
+#define AWQ_GEMV4_KS 4
 #endif
 
-// Consumer warps: 4 (two 16-row tiles each) up to M = 16; 8 (one tile each) above, where the
-// extra warps hide the longer mma chains (measured on the Llama-2-7B and 70B decode shapes).
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
   const int mt = (M + 7) / 8;
   switch (mt) {
     case 1:
-      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 2: return launch_gemv_cfg<2, 3, 4, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, AWQ_GEMV1_CW>(x, qw, sc, zr, y, M, N, K, dev, num_sms,
+                                                                             stream);
+    case 2:
+      return launch_gemv_cfg<2, AWQ_GEMV2_STAGES, AWQ_GEMV2_KS, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
     case 3: return launch_gemv_cfg<3, 3, 4, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    default: return launch_gemv_cfg<4, 4, 2, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default:
+      return launch_gemv_cfg<4, AWQ_GEMV4_STAGES, AWQ_GEMV4_KS, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   }
 }
 
