@@ -51,21 +51,72 @@ constexpr int kGemvNacc =
     MT == 2 ? 2 : 1;
 #endif
 
-// Adds one quantization group (two 64-k tiles) of a consumer warp's NT 16-row tiles to acc.
-//   xg: the group's two activation boxes in shared memory (8*MT tokens x 64 k fp16 each,
-//       128-byte swizzle, 1024 bytes per 8 tokens), back to back;
+// One quantization group (two 64-k tiles) of a consumer warp's fragments, in registers
+// (loaded from the stage right before the group's math):
+//   w[ii][n]     the lane's 16 bytes of codes of k-tile ii, 16-row tile n (packed layout v1:
+//                exactly the m16n8k16 A fragments of 4 k-steps for rows r, r+8);
+//   xv[ii][j][2] the lane's 32 bytes of x' of k-tile ii, token tile j (B fragments);
+//   sv[n], zz[n] the scale pair (rows r, r+8) and the zero-point byte of tile n;
+//   sx[2]        (kSumX) the group's activation sums of tokens 0 and 1.
+template <int MT, int NT>
+struct GemvGroupRegs {
+  uint4 w[2][NT];
+  uint4 xv[2][MT][2];
+  uint32_t sv[NT];
+  uint32_t zz[NT];
+  uint2 sx[2];   // raw fp16 quads for the activation sums (kSumX)
+};
+
+// Loads a group's fragments from the stage in shared memory.
+//   xg: the group's two activation boxes (8*MT tokens x 64 k fp16 each, 128-byte swizzle, 1024
+//       bytes per 8 tokens), back to back;
 //   wg: the group's two 4 KB super-chunks of packed codes, offset to the warp's first 16-row
 //       tile and to this lane's 16 bytes (each further tile is 512 bytes further);
 //   scg / zg: the warp's scales / zeros of the group, offset to this lane's fragment row r.
-// A operand: a code pair is masked out of the word and OR-ed into the mantissa of fp16 1024
-// (0x6400), giving 1024 + q (even nibbles) or 1024 + 16q (odd nibbles, which sit 4 bits
-// higher); subtracting 1024 + z, resp. 1024 + 16z, leaves q - z or 16 (q - z): small integers,
-// exact in fp16, so every tensor-core product x' (q - z) is exact. The group's fp32 sums are
-// then scaled by S (rows r) and S/16 (rows r+8, the odd nibbles).
-template <int MT, int NACC, int NT>
-__device__ __forceinline__ void gemv_group(float (&acc)[NT][MT][4], const uint8_t* xg, const uint8_t* wg,
-                                           const uint8_t* scg, const uint8_t* zg, int r, int t) {
+template <int MT, int NT, bool kSumX>
+__device__ __forceinline__ void gemv_group_load(GemvGroupRegs<MT, NT>& g, const uint8_t* xg, const uint8_t* wg,
+                                                const uint8_t* scg, const uint8_t* zg, int r, int t) {
   constexpr int kBox = 8 * MT * 128;
+#pragma unroll
+  for (int ii = 0; ii < 2; ++ii) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) g.w[ii][n] = *reinterpret_cast<const uint4*>(wg + ii * 4096 + n * 512);
+#pragma unroll
+    for (int j = 0; j < MT; ++j) {
+      const int m = 8 * j + r;
+      const uint8_t* row = xg + ii * kBox + m * 128;
+      g.xv[ii][j][0] = *reinterpret_cast<const uint4*>(row + (((2 * t) ^ (m & 7)) << 4));
+      g.xv[ii][j][1] = *reinterpret_cast<const uint4*>(row + (((2 * t + 1) ^ (m & 7)) << 4));
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    g.sv[n] = *reinterpret_cast<const uint32_t*>(scg + n * 32);
+    g.zz[n] = zg[n * 8];
+  }
+  if (kSumX) {
+    // tokens 0 and 1 of the group: lane l reads 4 values of k-tile l >> 4 at k = 4 (l & 15);
+    // box row 1 sits in 16-byte chunks swizzled by c ^ 1
+    const int lane = 4 * r + t;
+    const uint8_t* box = xg + (lane >> 4) * kBox;
+    const int c16 = (lane & 15) >> 1, off = (lane & 1) << 3;
+    g.sx[0] = *reinterpret_cast<const uint2*>(box + (c16 << 4) + off);
+    g.sx[1] = *reinterpret_cast<const uint2*>(box + 128 + ((c16 ^ 1) << 4) + off);
+  }
+}
+
+// Adds one group to acc. Two exact dequantizations:
+//  * kSumX == false (any M): a code pair is masked out of its word and OR-ed into the mantissa
+//    of fp16 1024 (0x6400), giving 1024 + q (even nibbles) or 1024 + 16q (odd nibbles, 4 bits
+//    higher); subtracting 1024 + z, resp. 1024 + 16z, leaves q - z or 16 (q - z), small
+//    integers exact in fp16. The group's fp32 sums are scaled by S and S/16.
+//  * kSumX == true (M <= 2): one AND per pair gives the codes as exact fp16 subnormals q 2^-24
+//    (16q 2^-24 for the odd nibbles), and the zero point enters once per group as
+//    -S z sum_k x'_mk, with the activation sums of tokens 0 and 1 added up by the warp
+//    (4 values per lane and a butterfly). The group's fp32 sums are scaled by S 2^24, S 2^20.
+// Either way every tensor-core product is exact.
+template <int MT, int NACC, int NT, bool kSumX>
+__device__ __forceinline__ void gemv_group_math(float (&acc)[NT][MT][4], const GemvGroupRegs<MT, NT>& g, int t) {
   float tq[NACC][NT][MT][4];
 #pragma unroll
   for (int a = 0; a < NACC; ++a)
@@ -76,40 +127,38 @@ __device__ __forceinline__ void gemv_group(float (&acc)[NT][MT][4], const uint8_
 #pragma unroll
         for (int c = 0; c < 4; ++c) tq[a][n][j][c] = 0.f;
   uint32_t zlo[NT], zhi[NT];   // fp16 pairs 1024 + z (row r) and 1024 + 16 z (row r+8)
+  if (!kSumX) {
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const uint32_t zz = zg[n * 8];
-    zlo[n] = 0x64006400u + (zz & 0xFu) * 0x00010001u;
-    zhi[n] = 0x64006400u + (zz >> 4) * 0x00100010u;
+    for (int n = 0; n < NT; ++n) {
+      zlo[n] = 0x64006400u + (g.zz[n] & 0xFu) * 0x00010001u;
+      zhi[n] = 0x64006400u + (g.zz[n] >> 4) * 0x00100010u;
+    }
   }
 #pragma unroll
   for (int ii = 0; ii < 2; ++ii) {
-    uint4 w[NT];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) w[n] = *reinterpret_cast<const uint4*>(wg + ii * 4096 + n * 512);
-    uint4 xv[MT][2];
-#pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      const int m = 8 * j + r;
-      const uint8_t* row = xg + ii * kBox + m * 128;
-      xv[j][0] = *reinterpret_cast<const uint4*>(row + (((2 * t) ^ (m & 7)) << 4));
-      xv[j][1] = *reinterpret_cast<const uint4*>(row + (((2 * t + 1) ^ (m & 7)) << 4));
-    }
 #pragma unroll
     for (int s4 = 0; s4 < 4; ++s4) {
       const int ac = (ii * 4 + s4) % NACC;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        const uint32_t q = (s4 == 0) ? w[n].x : (s4 == 1) ? w[n].y : (s4 == 2) ? w[n].z : w[n].w;
+        const uint4& wv = g.w[ii][n];
+        const uint32_t q = (s4 == 0) ? wv.x : (s4 == 1) ? wv.y : (s4 == 2) ? wv.z : wv.w;
         const uint32_t q8 = q >> 8;
         uint32_t a[4];
-        a[0] = hsub2_u32(lop_or(q, 0x000F000Fu, 0x64006400u), zlo[n]);    // row r,   e0 e1: q - z
-        a[1] = hsub2_u32(lop_or(q, 0x00F000F0u, 0x64006400u), zhi[n]);    // row r+8, e0 e1: 16 (q - z)
-        a[2] = hsub2_u32(lop_or(q8, 0x000F000Fu, 0x64006400u), zlo[n]);   // row r,   e2 e3
-        a[3] = hsub2_u32(lop_or(q8, 0x00F000F0u, 0x64006400u), zhi[n]);   // row r+8, e2 e3
+        if (kSumX) {
+          a[0] = q & 0x000F000Fu;     // row r,   slots e0 e1:  q * 2^-24
+          a[1] = q & 0x00F000F0u;     // row r+8, slots e0 e1: 16q * 2^-24
+          a[2] = q8 & 0x000F000Fu;    // row r,   slots e2 e3
+          a[3] = q8 & 0x00F000F0u;    // row r+8, slots e2 e3
+        } else {
+          a[0] = hsub2_u32(lop_or(q, 0x000F000Fu, 0x64006400u), zlo[n]);    // row r,   e0 e1: q - z
+          a[1] = hsub2_u32(lop_or(q, 0x00F000F0u, 0x64006400u), zhi[n]);    // row r+8, e0 e1: 16 (q - z)
+          a[2] = hsub2_u32(lop_or(q8, 0x000F000Fu, 0x64006400u), zlo[n]);   // row r,   e2 e3
+          a[3] = hsub2_u32(lop_or(q8, 0x00F000F0u, 0x64006400u), zhi[n]);   // row r+8, e2 e3
+        }
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
-          const uint4& xq = xv[j][s4 >> 1];
+          const uint4& xq = g.xv[ii][j][s4 >> 1];
           mma_m16n8k16_f32(tq[ac][n][j], a, (s4 & 1) ? xq.z : xq.x, (s4 & 1) ? xq.w : xq.y);
         }
       }
@@ -123,18 +172,42 @@ __device__ __forceinline__ void gemv_group(float (&acc)[NT][MT][4], const uint8_
       for (int j = 0; j < MT; ++j)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tq[0][n][j][c] += tq[a][n][j][c];
-  // end of the group: acc += S (sum x (q - z)); rows r+8 carry 16 (q - z)
+  if (kSumX) {
+    const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&g.sx[0].x));
+    const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&g.sx[0].y));
+    const float2 b0 = __half22float2(*reinterpret_cast<const __half2*>(&g.sx[1].x));
+    const float2 b1 = __half22float2(*reinterpret_cast<const __half2*>(&g.sx[1].y));
+    float sx0 = (a0.x + a0.y) + (a1.x + a1.y), sx1 = (b0.x + b0.y) + (b1.x + b1.y);
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const uint32_t sv = *reinterpret_cast<const uint32_t*>(scg + n * 32);
-    const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sv));
-    const float c_lo = sf.x, c_hi = sf.y * 0.0625f;
+    for (int o = 16; o > 0; o >>= 1) {
+      sx0 += __shfl_xor_sync(0xFFFFFFFFu, sx0, o);
+      sx1 += __shfl_xor_sync(0xFFFFFFFFu, sx1, o);
+    }
+    // acc element c holds token 2t + (c & 1); tokens >= 2 only exist for M > 2 (unused here)
 #pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      acc[n][j][0] = fmaf(c_lo, tq[0][n][j][0], acc[n][j][0]);
-      acc[n][j][1] = fmaf(c_lo, tq[0][n][j][1], acc[n][j][1]);
-      acc[n][j][2] = fmaf(c_hi, tq[0][n][j][2], acc[n][j][2]);
-      acc[n][j][3] = fmaf(c_hi, tq[0][n][j][3], acc[n][j][3]);
+    for (int n = 0; n < NT; ++n) {
+      const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&g.sv[n]));
+      const float c_lo = sf.x * 16777216.0f, c_hi = sf.y * 1048576.0f;
+      const float d_lo = -sf.x * static_cast<float>(g.zz[n] & 0xFu);
+      const float d_hi = -sf.y * static_cast<float>(g.zz[n] >> 4);
+      acc[n][0][0] = fmaf(d_lo, sx0, fmaf(c_lo, tq[0][n][0][0], acc[n][0][0]));
+      acc[n][0][1] = fmaf(d_lo, sx1, fmaf(c_lo, tq[0][n][0][1], acc[n][0][1]));
+      acc[n][0][2] = fmaf(d_hi, sx0, fmaf(c_hi, tq[0][n][0][2], acc[n][0][2]));
+      acc[n][0][3] = fmaf(d_hi, sx1, fmaf(c_hi, tq[0][n][0][3], acc[n][0][3]));
+    }
+  } else {
+    // acc += S (sum x (q - z)); rows r+8 carry 16 (q - z)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&g.sv[n]));
+      const float c_lo = sf.x, c_hi = sf.y * 0.0625f;
+#pragma unroll
+      for (int j = 0; j < MT; ++j) {
+        acc[n][j][0] = fmaf(c_lo, tq[0][n][j][0], acc[n][j][0]);
+        acc[n][j][1] = fmaf(c_lo, tq[0][n][j][1], acc[n][j][1]);
+        acc[n][j][2] = fmaf(c_hi, tq[0][n][j][2], acc[n][j][2]);
+        acc[n][j][3] = fmaf(c_hi, tq[0][n][j][3], acc[n][j][3]);
+      }
     }
   }
 }
@@ -160,7 +233,7 @@ struct GemvCfg {
   }
 };
 
-template <int MT, int S, int KS, int CW>
+template <int MT, int S, int KS, int CW, bool kSumX>
 __global__ void __launch_bounds__(GemvCfg<MT, S, KS, CW>::kThreads, 1) gemv_kernel(
     const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
     const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M, int N,
@@ -283,9 +356,12 @@ __global__ void __launch_bounds__(GemvCfg<MT, S, KS, CW>::kThreads, 1) gemv_kern
         const uint8_t* szr = sb + C::kX + C::kW + C::kSc + (NT * cw) * 8 + r;
 #pragma unroll
         for (int i = 0; i < KS; i += 2)
-          if (i < nk)
-            gemv_group<MT, kGemvNacc<MT>, NT>(acc, sb + i * C::kMP * 128, sw + i * 4096, ssc + (i / 2) * 256,
-                                              szr + (i / 2) * 64, r, t);
+          if (i < nk) {
+            GemvGroupRegs<MT, NT> gr;
+            gemv_group_load<MT, NT, kSumX>(gr, sb + i * C::kMP * 128, sw + i * 4096, ssc + (i / 2) * 256,
+                                           szr + (i / 2) * 64, r, t);
+            gemv_group_math<MT, kGemvNacc<MT>, NT, kSumX>(acc, gr, t);
+          }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == S) { stage = 0; phase ^= 1; }

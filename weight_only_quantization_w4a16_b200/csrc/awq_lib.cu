@@ -174,11 +174,12 @@ int max_active_clusters(Kernel kernel, int threads, size_t smem, int cl, int dev
   return n;
 }
 
-template <int MT, int S, int KS, int CW>
+template <int MT, int S, int KS, int CW, bool kSumX = false>
 awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
                              int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
   using Cfg = GemvCfg<MT, S, KS, CW>;
-  auto kernel = gemv_kernel<MT, S, KS, CW>;
+  static_assert(!kSumX || MT == 1, "activation sums are taken for tokens 0 and 1 only");
+  auto kernel = gemv_kernel<MT, S, KS, CW, kSumX>;
   constexpr int kMaxSmem = 227 * 1024;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
@@ -250,6 +251,11 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
   const int mt = (M + 7) / 8;
   switch (mt) {
     case 1:
+      // M <= 2: codes as fp16 subnormals (one AND per pair) and the zero point through the
+      // activation sums, which the warp takes from the activation box at little cost
+      if (M <= 2)
+        return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, AWQ_GEMV1_CW, true>(x, qw, sc, zr, y, M, N, K, dev,
+                                                                                     num_sms, stream);
       return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, AWQ_GEMV1_CW>(x, qw, sc, zr, y, M, N, K, dev, num_sms,
                                                                              stream);
     case 2:
