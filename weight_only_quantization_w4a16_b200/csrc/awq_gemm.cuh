@@ -50,7 +50,8 @@ struct GemmCfg {
   static constexpr int kNumBars = 3 * STAGES + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;        // + slack for 1024-byte alignment
-  static constexpr int kTmemCols = 2 * BT < 32 ? 32 : 2 * BT;
+  // two accumulators of BT columns; tcgen05.alloc takes a power of two >= 32 columns
+  static constexpr int kTmemCols = 2 * BT <= 32 ? 32 : 2 * BT <= 64 ? 64 : 2 * BT <= 128 ? 128 : 2 * BT <= 256 ? 256 : 512;
   static constexpr int kThreads = (NDQ + 6) * 32;
   static constexpr int kWarpEpi0 = NDQ;
   static constexpr int kWarpProd = NDQ + 4;

@@ -290,14 +290,25 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 
 awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  if (M <= 32) return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  if (M <= 64) return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  // Token tile by a round model: the persistent CTAs (one per SM) take tiles round-robin, so a
+  // launch costs ceil(tiles / SMs) rounds, and a tile's time grows only slowly with BT because
+  // dequantizing its 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted
+  // on the Llama-3-8B prefill and Llama-2-70B layers at M = 512 and 2048).
   const long long nst = padded_rows(N) / kSuperRows;
-  auto tiles = [&](int bt) { return nst * ((M + bt - 1) / bt); };
-  if (M > 128 && tiles(256) >= num_sms)
-    return launch_gemm_cfg<256, 4, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  if (M > 64 && tiles(128) >= (num_sms * 3) / 4)
-    return launch_gemm_cfg<128, 6, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  if (M > 32) return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  int best_bt = 64;
+  double best = 1e300;
+  for (int bt : {256, 128, 64}) {
+    const long long tiles = nst * ((M + bt - 1) / bt);
+    const double cost = static_cast<double>((tiles + num_sms - 1) / num_sms) * (0.75 + 0.35 * bt / 256.0);
+    if (cost < best - 1e-9) { best = cost; best_bt = bt; }
+  }
+  switch (best_bt) {
+    case 256: return launch_gemm_cfg<256, 4, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 128: return launch_gemm_cfg<128, 6, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default: return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  }
 }
 
 awq_status_t check_linear_args(const void* x, const void* qw, const void* sc, const void* zr, const void* y, int M,
