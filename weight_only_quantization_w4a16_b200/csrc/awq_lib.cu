@@ -283,15 +283,26 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
                    qw, sc, zr, y, M, N, K);
 }
 
-// Compile-time tuning of the prefill kernel: dequantization warps.
+// Compile-time tuning of the prefill kernel: dequantization warps, ring stages per token tile
+// (the deepest ring that fits in shared memory).
 #ifndef AWQ_GEMM_NDQ
 #define AWQ_GEMM_NDQ 8
+#endif
+#ifndef AWQ_GEMM_S256
+#define AWQ_GEMM_S256 4
+#endif
+#ifndef AWQ_GEMM_S128
+#define AWQ_GEMM_S128 6
+#endif
+#ifndef AWQ_GEMM_S64
+#define AWQ_GEMM_S64 7
 #endif
 
 awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
   if (M <= 32) return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  if (M <= 64) return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+  if (M <= 64)
+    return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   // Token tile by a round model: the persistent CTAs (one per SM) take tiles round-robin, so a
   // launch costs ceil(tiles / SMs) rounds, and a tile's time grows only slowly with BT because
   // dequantizing its 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted
@@ -304,10 +315,16 @@ awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, 
     const double cost = static_cast<double>((tiles + num_sms - 1) / num_sms) * (0.75 + 0.35 * bt / 256.0);
     if (cost < best - 1e-9) { best = cost; best_bt = bt; }
   }
+#ifdef AWQ_GEMM_FORCE_BT
+  best_bt = AWQ_GEMM_FORCE_BT;
+#endif
   switch (best_bt) {
-    case 256: return launch_gemm_cfg<256, 4, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 128: return launch_gemm_cfg<128, 6, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    default: return launch_gemm_cfg<64, 7, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 256:
+      return launch_gemm_cfg<256, AWQ_GEMM_S256, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 128:
+      return launch_gemm_cfg<128, AWQ_GEMM_S128, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default:
+      return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   }
 }
 
