@@ -142,7 +142,15 @@ AWQ_API awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scal
  *   x  fp16 [M, K] row-major (the scaled activations x'), 1 <= M <= 32.
  *   y  fp16 [M, N] row-major.
  * y = x . dequant^T with fp32 accumulation; dequant(q) = (q - z) * S.
- * Requires N >= 1, K >= 128, K % 128 == 0. */
+ * Bitwise reproducible from call to call. Requires N >= 1, K >= 128,
+ * K % 128 == 0.
+ * Weight prefetch: the kernel starts reading qweight, scales and zeros as soon
+ * as it is resident, which under programmatic dependent launch can be before
+ * the preceding kernel of `stream` has finished (x and y are touched only
+ * after it has). The packed weights must therefore be complete before that
+ * preceding kernel begins: true when they were written by an earlier kernel or
+ * copy, or by awq_quantize_g128, which lets no later kernel start before it
+ * has completed and its writes are visible. */
 AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                             const uint8_t* zeros, uint16_t* y, int M, int N, int K,
                             awq_stream_t stream);
@@ -155,7 +163,8 @@ AWQ_API awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, 
                             const uint8_t* zeros, uint16_t* y, int M, int N, int K,
                             awq_stream_t stream);
 
-/* Convenience dispatch: awq_w4a16_gemv for M <= 32, awq_w4a16_gemm otherwise. */
+/* Convenience dispatch: awq_w4a16_gemv for M <= 32 (same weight-prefetch
+ * rule), awq_w4a16_gemm otherwise. */
 AWQ_API awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                               const uint8_t* zeros, uint16_t* y, int M, int N, int K,
                               awq_stream_t stream);

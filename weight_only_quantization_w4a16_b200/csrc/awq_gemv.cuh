@@ -17,9 +17,12 @@
 //  * packed layout v1 makes each consumer lane's 16-byte read exactly the
 //    m16n8k16 A-fragments of 4 k-steps for rows r, r+8 of a 16-row tile, and
 //    the matching activation slots a contiguous 32-byte run of x' per token;
-//  * dequantization is two instructions per code pair (LOP3 into the fp16
-//    mantissa of 1024, HSUB2 of 1024 + z) and yields q - z exactly, so every
-//    tensor-core product is exact; S is applied in fp32 to each group's sums;
+//  * dequantization yields exact small integers, so every tensor-core product
+//    is exact: for M >= 3 two instructions per code pair (LOP3 into the fp16
+//    mantissa of 1024, HSUB2 of 1024 + z) give q - z; for M <= 2 one AND per
+//    pair gives q as an fp16 subnormal and the zero point is applied per
+//    group through the activation sums; S is applied in fp32 to each group's
+//    sums;
 //  * persistent clusters: cluster c walks super-tiles c, c + C, ...; its CL
 //    CTAs split K and keep every super-tile's partial sums in shared memory,
 //    so the stream never stops for a barrier; one cluster barrier at the end
@@ -42,7 +45,7 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Independent accumulator chains per 16-row tile in gemv_group (shorter dependent-mma chains).
+// Independent accumulator chains per 16-row tile in gemv_group_math (shorter dependent-mma chains).
 template <int MT>
 constexpr int kGemvNacc =
 #ifdef AWQ_GEMV_NACC

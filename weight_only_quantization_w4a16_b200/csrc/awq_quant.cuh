@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
   }
   __syncthreads();
   // Wait for the previous kernel, but do not let the next one start early: kernels that read
-  // packed weights before their own wait (the split-K decode kernel) may follow, so the next
+  // packed weights before their own wait (the decode kernel) may follow, so the next
   // kernel launches only once this grid has completed and every write below is visible.
   pdl_wait();
   const unsigned long long budget = g_wait_budget_ns;
