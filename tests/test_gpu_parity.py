@@ -245,3 +245,49 @@ def test_prefill_full_size_sampled(layer_idx, M):
 def test_70b_full_size_sampled(layer_idx, M, fn):
     _full_size_case("llama2_70b_layers", layer_idx, M, fn)
 
+
+
+# ----------------------------------------------------------------------------- launch chaining
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_decode_chained_on_requantized_buffers(use_graph):
+    """a1 -> a2 -> a3 for three different layers into the SAME packed buffers, launched back to back
+    on one stream with no host synchronization (eagerly, and captured in a CUDA graph, which keeps
+    programmatic dependent launch). Each decode reads weights that the immediately preceding
+    quantizer wrote, and each quantizer overwrites weights the previous decode read: the decode
+    kernel's early weight reads must still see complete, current weights."""
+    P = lib()
+    torch = torch_mod()
+    N, K = 2048, 4096
+    cases = [workloads.random_case(121 + i, 1 + i, N, K) for i in range(3)]
+    dx = [dev(x) for x, _ in cases]
+    dW = [dev(W) for _, W in cases]
+    packed = P.alloc_packed(N, K)
+    s = [torch.empty(K, dtype=torch.float32, device="cuda") for _ in cases]
+    xs = [torch.empty_like(x) for x in dx]
+    ys = [torch.empty((x.shape[0], N), dtype=torch.float16, device="cuda") for x in dx]
+
+    def chain():
+        for i in range(len(cases)):
+            P.awq_activation_scale(dx[i], 0.5, s[i], xs[i])
+            P.awq_quantize_g128(dW[i], s[i], packed)
+            P.awq_w4a16_gemv(xs[i], *packed, N, ys[i])
+
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        chain()   # eager run (also sets kernel attributes before any capture)
+        if use_graph:
+            for y in ys:
+                y.zero_()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                chain()
+            g.replay()
+        stream.synchronize()
+    assert P.awq_poll_device_status() == P.AWQ_OK
+    for i, (x, W) in enumerate(cases):
+        r = O.reference_forward(x, W)
+        if i == len(cases) - 1:   # the buffers hold the last layer's codes
+            assert np.array_equal(host(packed[0]).view(np.uint32), O.pack(r["q"], r["S"], r["z"])[0])
+        y = host(ys[i]).astype(np.float64)
+        assert_tolerance(y, r["y"], f"chained layer {i}")
+        assert_tight(y, r["y"], what=f"chained layer {i}")
