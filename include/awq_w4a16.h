@@ -27,7 +27,8 @@
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers owned by the caller. The library
  *     allocates no memory and never synchronizes, except awq_poll_device_status
- *     and awq_debug_set_wait_budget_ns, which say so.
+ *     and the test hooks awq_debug_set_wait_budget_ns and
+ *     awq_debug_drop_first_copy, which say so.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream) and runs asynchronously; outputs are valid once the stream reaches
  *     that point.
