@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -274,11 +275,17 @@ def bench_config(wl, M):
 
 # ----------------------------------------------------------------------------- ours
 def kernel_source_hash(name):
+    """SHA-256 (first 16 hex digits) of a kernel source with comments and whitespace removed, so
+    that only a change of the code itself invalidates a recorded profile."""
     p = os.path.join(ROOT, "weight_only_quantization_w4a16_b200", "csrc", name)
     try:
-        return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+        src = open(p).read()
     except OSError:
         return None
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    src = re.sub(r"\s+", "", src)
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
 def profile_traffic(kernel_file, workload, M):
