@@ -30,9 +30,13 @@
 
 namespace awq {
 
-template <int BT, int STAGES, int NDQ>
+// CPS: resident CTAs per SM. With 2, each CTA keeps one TMEM accumulator (the other CTA's
+// epilogue and mainloop interleave with its own); with 1, two accumulators let the epilogue of
+// one tile overlap the mainloop of the next.
+template <int BT, int STAGES, int NDQ, int CPS = 1>
 struct GemmCfg {
   static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
+  static_assert(CPS == 1 || CPS == 2, "CTAs per SM");
   static_assert(NDQ == 4 || NDQ == 8, "dequant warps");
   static constexpr int kA = kSuperRows * kKTile * 2;        // 16 KB dequantized weights
   static constexpr int kB = BT * kKTile * 2;                // x' tile
@@ -51,20 +55,25 @@ struct GemmCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;        // + slack for 1024-byte alignment
   // two accumulators of BT columns; tcgen05.alloc takes a power of two >= 32 columns
-  static constexpr int kTmemCols = 2 * BT <= 32 ? 32 : 2 * BT <= 64 ? 64 : 2 * BT <= 128 ? 128 : 2 * BT <= 256 ? 256 : 512;
+  static constexpr int kNAcc = CPS == 2 ? 1 : 2;   // TMEM accumulators of BT columns
+  // tcgen05.alloc takes a power of two >= 32 columns; all CTAs of an SM share its 512
+  static constexpr int kTmemCols = kNAcc * BT <= 32 ? 32 : kNAcc * BT <= 64 ? 64 : kNAcc * BT <= 128 ? 128
+                                   : kNAcc * BT <= 256 ? 256 : 512;
+  static_assert(kTmemCols * CPS <= 512, "tensor memory");
   static constexpr int kThreads = (NDQ + 6) * 32;
   static constexpr int kWarpEpi0 = NDQ;
   static constexpr int kWarpProd = NDQ + 4;
   static constexpr int kWarpMma = NDQ + 5;
   static_assert(kSmem <= 232448, "shared memory");
+  static_assert(CPS == 1 || (kSmem + 1024) * 2 <= 233472, "two CTAs per SM must fit in shared memory");
 };
 
-template <int BT, int STAGES, int NDQ>
-__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ>::kThreads, 1)
+template <int BT, int STAGES, int NDQ, int CPS>
+__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
                 const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
                 int N, int K) {
-  using C = GemmCfg<BT, STAGES, NDQ>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -152,8 +161,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ>::kThreads, 1)
       bool ok = true, any = false;
       int it = 0;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
-        const int b = it & 1;
-        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        const int b = it % C::kNAcc;
+        const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
         if (!mbar_wait_bounded(&accempty[b], (use & 1) ^ 1, s_abort, budget)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BT);
@@ -231,8 +240,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ>::kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
       const int st = tile % NST, mt = tile / NST;
-      const int b = it & 1;
-      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int b = it % C::kNAcc;
+      const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
       if (!mbar_wait_bounded(&accfull[b], use & 1, s_abort, budget)) { ok = false; break; }
       tc_fence_after();
       const int n = st * kSuperRows + 32 * e + lane;

@@ -267,20 +267,21 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
-template <int BT, int STAGES, int NDQ>
+template <int BT, int STAGES, int NDQ, int CPS = 1>
 awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
                              int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using C = GemmCfg<BT, STAGES, NDQ>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS>;
+  auto kernel = gemm_kernel<BT, STAGES, NDQ, CPS>;
   static std::atomic<uint64_t> smem_done{0};
-  awq_status_t st = ensure_smem(gemm_kernel<BT, STAGES, NDQ>, C::kSmem, dev, smem_done);
+  awq_status_t st = ensure_smem(kernel, C::kSmem, dev, smem_done);
   if (st != AWQ_OK) return st;
   CUtensorMap map;
   st = make_x_map(&map, x, M, K, BT);
   if (st != AWQ_OK) return st;
   const long long tiles = static_cast<long long>(padded_rows(N) / kSuperRows) * ((M + BT - 1) / BT);
-  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms));
-  return launch_ex(gemm_kernel<BT, STAGES, NDQ>, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), 0, C::kSmem, stream, map,
-                   qw, sc, zr, y, M, N, K);
+  const int grid = static_cast<int>(std::min<long long>(tiles, static_cast<long long>(CPS) * num_sms));
+  return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), 0, C::kSmem, stream, map, qw, sc, zr, y, M, N,
+                   K);
 }
 
 // Compile-time tuning of the prefill kernel: dequantization warps, ring stages per token tile
