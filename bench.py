@@ -274,18 +274,22 @@ def bench_config(wl, M):
 
 
 # ----------------------------------------------------------------------------- ours
-def kernel_source_hash(name):
-    """SHA-256 (first 16 hex digits) of a kernel source with comments and whitespace removed, so
-    that only a change of the code itself invalidates a recorded profile."""
-    p = os.path.join(ROOT, "weight_only_quantization_w4a16_b200", "csrc", name)
-    try:
-        src = open(p).read()
-    except OSError:
-        return None
+def code_hash(src):
+    """SHA-256 (first 16 hex digits) of C++/CUDA source text with comments and whitespace removed,
+    so that only a change of the code itself counts."""
     src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
     src = re.sub(r"//[^\n]*", " ", src)
     src = re.sub(r"\s+", "", src)
     return hashlib.sha256(src.encode()).hexdigest()[:16]
+
+
+def kernel_source_hash(name):
+    """code_hash of a kernel source file of the package (None if it is missing)."""
+    p = os.path.join(ROOT, "weight_only_quantization_w4a16_b200", "csrc", name)
+    try:
+        return code_hash(open(p).read())
+    except OSError:
+        return None
 
 
 def profile_traffic(kernel_file, workload, M):
