@@ -40,20 +40,26 @@
  *   - Only device ordinals with compute capability 10.0 are supported
  *     (AWQ_ERR_UNSUPPORTED otherwise).
  *
- * Packed layout, version 1 (awq_layout_version() == 1).
- *   Rows are padded to Np = ceil(N/128)*128 (padding rows: code 0, scale 0,
- *   zero 0). With
- *     n = st*128 + nt*16 + h*8 + r        (st super-tile, nt 16-row tile, h half, r row)
- *     k = kt*64 + t*16 + s*4 + e1*2 + e0  (kt 64-k tile, t column block, s step, e slot)
- *     g = k / 128,  KT = K/64,  G = K/128
- *   qweight: uint32[Np*K/8];  code q[n][k] sits in word
- *            ((st*KT + kt)*8 + nt)*128 + (4*r + t)*4 + s,  nibble h + 2*e1 + 4*e0
+ * Packed layout, version 2 (awq_layout_version() == 2): "tile-major".
+ *   Rows are grouped in 16-row tiles, Ntiles = ceil(N/16). Along K the
+ *   groups are padded to an even count: G = K/128, G2 = ceil(G/2) group
+ *   pairs, KTp = 4*G2 64-k tiles per tile. Padding rows and padding groups
+ *   hold code 0, scale 0, zero 0. With
+ *     n = 16*T + 8*h + r                  (T tile, h half, r row)
+ *     k = 64*kt + 16*t + 4*s + 2*e1 + e0  (kt 64-k tile, t column block, s step, e slot)
+ *     g = k / 128
+ *   qweight: uint32[Ntiles*KTp*128];  code q[n][k] sits in word
+ *            (T*KTp + kt)*128 + (4*r + t)*4 + s,  nibble h + 2*e1 + 4*e0
  *            (bits 4*nibble .. 4*nibble+3).  The 16 bytes of words
  *            (.., 4r+t, 0..3) are exactly the m16n8k16 A-fragments of one lane
  *            (rows r, r+8; k in [16t, 16t+16) of a 64-k tile).
- *   scales:  fp16[Np*K/128]; S[n][g] at ((st*G + g)*8 + nt)*16 + 2*r + h
- *   zeros:   uint8[Np*K/256]; z[n][g] in byte ((st*G + g)*8 + nt)*8 + r,
+ *   scales:  fp16[Ntiles*2*G2*16]; S[n][g] at (T*2*G2 + g)*16 + 2*r + h
+ *   zeros:   uint8[Ntiles*2*G2*8]; z[n][g] in byte (T*2*G2 + g)*8 + r,
  *            low nibble for h = 0, high nibble for h = 1.
+ *   So one tile and group pair is 2048 bytes of codes, 64 of scales and 16
+ *   of zeros, and each tile's codes, scales and zeros run contiguously along
+ *   K: a range of (tile, group pair) items is one contiguous byte range of
+ *   each array.
  *   Base pointers of qweight, scales, zeros, x, x' and y must be 16-byte aligned.
  */
 #ifndef AWQ_W4A16_H_
@@ -96,8 +102,9 @@ AWQ_API const char* awq_status_string(int status);
  * AWQ_ERR_UNSUPPORTED otherwise. Pure host function. */
 AWQ_API awq_status_t awq_check_config(int bits, int group_size, int zero_point);
 
-/* Sizes in bytes of the packed arrays for an N x K layer (0 if N < 1,
- * K < 128 or K % 128 != 0). Pure host functions. */
+/* Sizes in bytes of the packed arrays for an N x K layer: Ntiles*G2 times
+ * 2048 (qweight), 64 (scales) and 16 (zeros). 0 if N < 1, N > 2^31 - 128,
+ * K < 128, K % 128 != 0 or 16*Ntiles*K > 2^34. Pure host functions. */
 AWQ_API size_t awq_qweight_bytes(int N, int K);
 AWQ_API size_t awq_scales_bytes(int N, int K);
 AWQ_API size_t awq_zeros_bytes(int N, int K);
@@ -129,7 +136,7 @@ AWQ_API awq_status_t awq_scale_activations(const uint16_t* x, const float* s, in
  * --q_backend real; HF config zero_point true).
  *   W          fp16 [N, K] row-major (device).
  *   fold_scale fp32 [K] (device) or NULL (= all ones, no fold).
- *   qweight, scales, zeros: outputs in packed layout v1, sizes from awq_*_bytes.
+ *   qweight, scales, zeros: outputs in packed layout v2, sizes from awq_*_bytes.
  * Codes, scales and zeros are bit-identical to the rules in the file header
  * (every step IEEE fp32, round to nearest even). Requires N >= 1, K >= 128,
  * K % 128 == 0. Values with |W*s| >= 65520 overflow fp16 to inf; the result is

@@ -40,7 +40,9 @@ Readings where the pages are silent (each is also listed in the design notes):
   are computed against the stored fp16 S;
 * zero z = clamp(rint(-lo / S), 0, 15), codes q = clamp(rint(w' / S) + z, 0, 15),
   rint = round half to even, fp32 division;
-* dequantization ŵ = (q - z) * S, exact in float64; y = x' . ŵ^T in float64.
+* dequantization ŵ = (q - z) * S, exact in float64; y = x' . ŵ^T in float64;
+* scale search: an even grid of 20 exponents over [0, 1); the squared Frobenius
+  error of the layer output on the calibration rows, against x . W^T, picks one.
 
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``
 (brute force, closed forms, invariants, exact rational arithmetic,
@@ -57,7 +59,6 @@ GROUP_SIZE = 128
 QMAX = (1 << BITS) - 1          # 15
 RANGE_FLOOR = np.float32(1e-5)  # floor on hi - lo (a constant group would divide by zero)
 MEAN_FLOOR = 1e-8               # floor on the mean |x| before the power
-SUPER_ROWS = 128                # rows per super-tile of the packed layout
 K_TILE = 64                     # k per packed tile
 
 
@@ -200,73 +201,125 @@ def check_tolerance(y: np.ndarray, y_ref: np.ndarray, rel_fro: float = 2e-3, max
 
 
 # --------------------------------------------------------------------------
-# Packed layout, version 1 (restated from its written specification)
+# AWQ scale search (the exponent alpha of the activation statistic)
+# --------------------------------------------------------------------------
+def alpha_grid(n_grid: int = 20) -> np.ndarray:
+    """Candidate exponents alpha_i = i / n_grid, i = 0 .. n_grid - 1 (float32 values).
+
+    [AWQ-README] "Usage" step 1 runs an AWQ search that picks the scales and
+    dumps them; [CSDN-AWQ] "02.02 AWQ" says the scales come from offline
+    activation statistics with no backpropagation. The pages give neither the
+    grid nor its size; reading: an even grid over [0, 1) of 20 points.
+    """
+    return (np.arange(n_grid, dtype=np.float64) / n_grid).astype(np.float32)
+
+
+def search_errors(x: np.ndarray, W: np.ndarray, alphas) -> np.ndarray:
+    """Squared output error of the whole path for every candidate alpha, float64.
+
+    For each alpha: s = activation_scale(x, alpha), x' = scale_activations(x, s),
+    w_hat = dequantize(quantize_groups(fold_weights(W, s))), and
+    err = || x . W^T - x' . w_hat^T ||_F^2 with both products in float64 over the
+    fp16 inputs (the layer's own output on the calibration rows is the target).
+    """
+    y_ref = np.asarray(x, np.float16).astype(np.float64) @ np.asarray(W, np.float16).astype(np.float64).T
+    errs = []
+    for a in alphas:
+        s = activation_scale(x, float(a))
+        y = linear(scale_activations(x, s), fake_quantize(W, s))
+        errs.append(float(np.sum((y - y_ref) ** 2)))
+    return np.array(errs, dtype=np.float64)
+
+
+def search_alpha(x: np.ndarray, W: np.ndarray, n_grid: int = 20):
+    """The grid point with the smallest squared output error (the first one on ties).
+
+    Returns (alpha, s, errors): the chosen exponent, its scale s[K] and the error of
+    every grid point.
+    """
+    alphas = alpha_grid(n_grid)
+    errs = search_errors(x, W, alphas)
+    i = int(np.argmin(errs))
+    return float(alphas[i]), activation_scale(x, float(alphas[i])), errs
+
+
+# --------------------------------------------------------------------------
+# Packed layout, version 2 (restated from its written specification)
 # --------------------------------------------------------------------------
 #
-# Rows are padded to Np = ceil(N / 128) * 128; padding rows hold code 0,
-# scale 0 and zero 0.  Index names:
-#   n = st*128 + nt*16 + h*8 + r        (super-tile st, 16-row tile nt, half h, row r)
-#   k = kt*64 + t*16 + s*4 + e1*2 + e0  (64-k tile kt, lane column t, step s, slot e)
+# Rows are grouped in 16-row tiles T (Ntiles = ceil(N / 16)); along K the
+# groups are padded to an even count (G2 = ceil(G / 2) group pairs,
+# KTp = 4 * G2 64-k tiles per tile).  Padding rows and padding groups hold
+# code 0, scale 0 and zero 0.  Index names:
+#   n = 16*T + 8*h + r                  (tile T, half h, row r)
+#   k = 64*kt + 16*t + 4*s + 2*e1 + e0  (64-k tile kt, lane column t, step s, slot e)
 #   g = k // 128
-# qweight (uint32, Np*K/8 words):
-#   word   = ((st*KT + kt)*8 + nt)*128 + (4*r + t)*4 + s,   KT = K/64
+# qweight (uint32, Ntiles*KTp*128 words):
+#   word   = (T*KTp + kt)*128 + (4*r + t)*4 + s
 #   nibble = h + 2*e1 + 4*e0  (bits 4*nibble .. 4*nibble+3)
-# scales (fp16, Np*K/128):  index ((st*G + g)*8 + nt)*16 + 2*r + h
-# zeros  (uint8, Np*K/256): byte  ((st*G + g)*8 + nt)*8 + r, low nibble h=0, high nibble h=1
+# scales (fp16, Ntiles*2*G2*16):  index (T*2*G2 + g)*16 + 2*r + h
+# zeros  (uint8, Ntiles*2*G2*8):  byte  (T*2*G2 + g)*8 + r, low nibble h=0, high nibble h=1
+# So every tile's codes, scales and zeros each run contiguously along K.
+TILE_ROWS = 16
+
+
+def layout_dims(N: int, K: int):
+    """(Ntiles, G, G2, KTp) of an N x K layer."""
+    G = K // GROUP_SIZE
+    G2 = -(-G // 2)
+    return -(-N // TILE_ROWS), G, G2, 4 * G2
+
+
 def padded_rows(N: int) -> int:
-    return -(-N // SUPER_ROWS) * SUPER_ROWS
+    return layout_dims(N, GROUP_SIZE)[0] * TILE_ROWS
 
 
 def pack(q: np.ndarray, S: np.ndarray, z: np.ndarray):
     """Codes/scales/zeros in plain [N, K] / [N, G] form -> (qweight, scales, zeros)."""
     N, K = q.shape
-    G = K // GROUP_SIZE
-    Np = padded_rows(N)
-    ST, KT = Np // SUPER_ROWS, K // K_TILE
-    qp = np.zeros((Np, K), dtype=np.uint32)
-    qp[:N] = q
-    # axes: st, nt, h, r, kt, t, s, e1, e0
-    a = qp.reshape(ST, 8, 2, 8, KT, 4, 4, 2, 2)
-    # word order (st, kt, nt, r, t, s); nibble order (e0, e1, h) -> nibble = 4*e0 + 2*e1 + h
-    a = a.transpose(0, 4, 1, 3, 5, 6, 8, 7, 2).reshape(-1, 8)
+    NT, G, G2, KTp = layout_dims(N, K)
+    qp = np.zeros((NT * TILE_ROWS, KTp * K_TILE), dtype=np.uint32)
+    qp[:N, :K] = q
+    # axes: T, h, r, kt, t, s, e1, e0
+    a = qp.reshape(NT, 2, 8, KTp, 4, 4, 2, 2)
+    # word order (T, kt, r, t, s); nibble order (e0, e1, h) -> nibble = 4*e0 + 2*e1 + h
+    a = a.transpose(0, 3, 2, 4, 5, 7, 6, 1).reshape(-1, 8)
     shifts = (4 * np.arange(8)).astype(np.uint32)
     qweight = np.bitwise_or.reduce(a << shifts, axis=1).astype(np.uint32)
 
-    Sp = np.zeros((Np, G), dtype=np.float16)
-    Sp[:N] = S
-    scales = Sp.reshape(ST, 8, 2, 8, G).transpose(0, 4, 1, 3, 2).reshape(-1).copy()
+    Sp = np.zeros((NT * TILE_ROWS, 2 * G2), dtype=np.float16)
+    Sp[:N, :G] = S
+    scales = Sp.reshape(NT, 2, 8, 2 * G2).transpose(0, 3, 2, 1).reshape(-1).copy()   # T, g, r, h
 
-    zp = np.zeros((Np, G), dtype=np.uint8)
-    zp[:N] = z
-    zz = zp.reshape(ST, 8, 2, 8, G).transpose(0, 4, 1, 3, 2)   # st, g, nt, r, h
+    zp = np.zeros((NT * TILE_ROWS, 2 * G2), dtype=np.uint8)
+    zp[:N, :G] = z
+    zz = zp.reshape(NT, 2, 8, 2 * G2).transpose(0, 3, 2, 1)                          # T, g, r, h
     zeros = (zz[..., 0] | (zz[..., 1] << 4)).astype(np.uint8).reshape(-1)
     return qweight, scales, zeros
 
 
 def unpack(qweight: np.ndarray, scales: np.ndarray, zeros: np.ndarray, N: int, K: int):
     """Inverse of ``pack``: (qweight, scales, zeros) -> (q[N, K], S[N, G], z[N, G])."""
-    G = K // GROUP_SIZE
-    Np = padded_rows(N)
-    ST, KT = Np // SUPER_ROWS, K // K_TILE
+    NT, G, G2, KTp = layout_dims(N, K)
     words = np.asarray(qweight, dtype=np.uint32).reshape(-1)
-    if words.size != Np * K // 8:
+    if words.size != NT * KTp * 128:
         raise ValueError("qweight has the wrong size")
     shifts = (4 * np.arange(8)).astype(np.uint32)
     nib = ((words[:, None] >> shifts) & np.uint32(0xF)).astype(np.uint8)
-    # nib axes: st, kt, nt, r, t, s, e0, e1, h -> back to st, nt, h, r, kt, t, s, e1, e0
-    a = nib.reshape(ST, KT, 8, 8, 4, 4, 2, 2, 2).transpose(0, 2, 8, 3, 1, 4, 5, 7, 6)
-    q = a.reshape(Np, K)[:N].copy()
+    # nib axes: T, kt, r, t, s, e0, e1, h -> back to T, h, r, kt, t, s, e1, e0
+    a = nib.reshape(NT, KTp, 8, 4, 4, 2, 2, 2).transpose(0, 7, 2, 1, 3, 4, 6, 5)
+    q = a.reshape(NT * TILE_ROWS, KTp * K_TILE)[:N, :K].copy()
 
-    sc = np.asarray(scales, dtype=np.float16).reshape(ST, G, 8, 8, 2)  # st, g, nt, r, h
-    S = sc.transpose(0, 2, 4, 3, 1).reshape(Np, G)[:N].copy()
+    sc = np.asarray(scales, dtype=np.float16).reshape(NT, 2 * G2, 8, 2)   # T, g, r, h
+    S = sc.transpose(0, 3, 2, 1).reshape(NT * TILE_ROWS, 2 * G2)[:N, :G].copy()
 
-    zb = np.asarray(zeros, dtype=np.uint8).reshape(ST, G, 8, 8)         # st, g, nt, r
-    zz = np.stack([zb & 0xF, zb >> 4], axis=-1)                        # st, g, nt, r, h
-    z = zz.transpose(0, 2, 4, 3, 1).reshape(Np, G)[:N].copy()
+    zb = np.asarray(zeros, dtype=np.uint8).reshape(NT, 2 * G2, 8)          # T, g, r
+    zz = np.stack([zb & 0xF, zb >> 4], axis=-1)                           # T, g, r, h
+    z = zz.transpose(0, 3, 2, 1).reshape(NT * TILE_ROWS, 2 * G2)[:N, :G].copy()
     return q, S, z
 
 
 def packed_sizes(N: int, K: int):
     """(qweight words, scale halves, zero bytes) for an N x K layer."""
-    Np = padded_rows(N)
-    return Np * K // 8, Np * K // GROUP_SIZE, Np * K // (2 * GROUP_SIZE)
+    NT, G, G2, KTp = layout_dims(N, K)
+    return NT * KTp * 128, NT * 2 * G2 * 16, NT * 2 * G2 * 8

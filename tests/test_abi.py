@@ -50,7 +50,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_layout_version_and_status_strings(lib):
-    assert lib.awq_layout_version() == 1
+    assert lib.awq_layout_version() == 2
     for code in range(6):
         s = lib.awq_status_string(code).decode()
         assert s.startswith("AWQ_")
@@ -75,7 +75,8 @@ def test_packed_sizes_match_layout_spec(lib, N, K):
     assert lib.awq_zeros_bytes(N, K) == zb
 
 
-@pytest.mark.parametrize("N,K", [(0, 128), (16, 0), (16, 100), (16, 192), (-1, 128)])
+@pytest.mark.parametrize("N,K", [(0, 128), (16, 0), (16, 100), (16, 192), (-1, 128), (2147483647, 128),
+                                 (2147483521, 128), (2 ** 30, 256)])
 def test_packed_sizes_reject_bad_shapes(lib, N, K):
     assert lib.awq_qweight_bytes(N, K) == 0 and lib.awq_scales_bytes(N, K) == 0 and lib.awq_zeros_bytes(N, K) == 0
 
@@ -100,6 +101,11 @@ def test_argument_checks_fail_before_any_device_call(lib):
     assert lib.awq_w4a16_gemm(V(A), V(A), V(A), V(A), V(A), 4, 16, 192, None) == 1
     assert lib.awq_activation_scale(V(A), 1, 12, 0.5, V(A), None, None) == 1
     assert lib.awq_activation_scale(V(A), 1, 128, float("nan"), V(A), None, None) == 1
+    # row counts whose padding would overflow an int, and layers past 2^34 packed weights
+    assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(A), 1, 2147483647, 128, None) == 1
+    assert lib.awq_w4a16_gemm(V(A), V(A), V(A), V(A), V(A), 64, 2147483600, 128, None) == 1
+    assert lib.awq_quantize_g128(V(A), None, 2147483647, 128, V(A), V(A), V(A), None) == 1
+    assert lib.awq_w4a16_linear(V(A), V(A), V(A), V(A), V(A), 1, 2 ** 27, 256, None) == 1
     # misaligned pointers
     assert lib.awq_quantize_g128(V(MIS), None, 16, 128, V(A), V(A), V(A), None) == 3
     assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(MIS), 1, 16, 128, None) == 3

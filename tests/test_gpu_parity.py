@@ -113,22 +113,33 @@ def test_quantize_hand_groups_and_extremes():
     _quant_check(W, s, W.shape[0], 256)
 
 
-def test_quantize_full_size_sampled():
-    """Llama-2-70B gate/up (N=28672, K=8192) with the AWQ fold: five sampled super-tiles."""
+def _full_layer_quant_check(W, s, rows_per_chunk=2048):
+    """Quantize a whole layer on the GPU; compare every packed byte with the oracle's codes packed by
+    the oracle's packer, chunk by chunk of rows (a tile's codes, scales and zeros are contiguous)."""
     P = lib()
-    wl = workloads.WORKLOADS["llama2_70b_layers"]
-    x, W = workloads.layer_inputs(wl, 0, 1)
     N, K = W.shape
-    s = O.activation_scale(x)
-    qw, sc, zb = P.awq_quantize_g128(dev(W), dev(s))
-    qw, sc, zb = host(qw).view(np.uint32), host(sc), host(zb)
-    KT, G = K // 64, K // 128
-    for st in [0, 1, 97, 150, N // 128 - 1]:
-        rows = slice(st * 128, st * 128 + 128)
-        q, S, z = O.unpack(qw[st * KT * 1024:(st + 1) * KT * 1024], sc[st * G * 128:(st + 1) * G * 128],
-                           zb[st * G * 64:(st + 1) * G * 64], 128, K)
-        q_ref, S_ref, z_ref = O.quantize_groups(O.fold_weights(W[rows], s))
-        assert np.array_equal(q, q_ref) and np.array_equal(f16_bits(S), f16_bits(S_ref)) and np.array_equal(z, z_ref)
+    qw, sc, zb = P.awq_quantize_g128(dev(W), dev(s) if s is not None else None)
+    qw, sc, zb = host(qw).view(np.uint32), f16_bits(host(sc)), host(zb)
+    _, _, G2, KTp = O.layout_dims(N, K)
+    for r0 in range(0, N, rows_per_chunk):
+        r1 = min(N, r0 + rows_per_chunk)
+        t0, t1 = r0 // 16, -(-r1 // 16)
+        q_ref, S_ref, z_ref = O.pack(*O.quantize_groups(O.fold_weights(W[r0:r1], s)))
+        assert np.array_equal(qw[t0 * KTp * 128:t1 * KTp * 128], q_ref), f"codes, rows {r0}..{r1}"
+        assert np.array_equal(sc[t0 * 2 * G2 * 16:t1 * 2 * G2 * 16], f16_bits(S_ref)), f"scales, rows {r0}..{r1}"
+        assert np.array_equal(zb[t0 * 2 * G2 * 8:t1 * 2 * G2 * 8], z_ref), f"zeros, rows {r0}..{r1}"
+
+
+@pytest.mark.parametrize("wl_name,li", [("llama2_70b_layers", 0), ("llama2_70b_layers", 1),
+                                        ("llama2_7b_decode_m1", 0), ("llama2_7b_decode_m1", 1),
+                                        ("llama2_7b_decode_m1", 2), ("llama2_7b_decode_m1", 3),
+                                        ("llama3_8b_prefill", 0), ("llama3_8b_prefill", 2),
+                                        ("llama3_8b_prefill", 3)])
+def test_quantize_full_layer_bit_exact(wl_name, li):
+    """Every packed byte of a full-size layer (with the AWQ fold from that layer's activations)."""
+    wl = workloads.WORKLOADS[wl_name]
+    x, W = workloads.layer_inputs(wl, li, wl.Ms[0])
+    _full_layer_quant_check(W, O.activation_scale(x))
 
 
 # ----------------------------------------------------------------------------- a3 / a4

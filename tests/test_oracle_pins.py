@@ -288,31 +288,32 @@ def test_fold_none_is_identity():
 # ----------------------------------------------------------------------------
 def test_layout_hand_positions():
     fx = _load("layout_positions.json")
-    N, K = fx["N"], fx["K"]
-    G = K // 128
-    words, nsc, nzb = O.packed_sizes(N, K)
-    assert (words, nsc, nzb) == (fx["sizes"]["words"], fx["sizes"]["scales"], fx["sizes"]["zero_bytes"])
-    for c in fx["codes"]:
-        q = np.zeros((N, K), np.uint8)
-        q[c["n"], c["k"]] = 0xB
-        qw, _, _ = O.pack(q, np.zeros((N, G), np.float16), np.zeros((N, G), np.uint8))
-        nz = np.nonzero(qw)[0]
-        assert nz.tolist() == [c["word"]]
-        assert int(qw[c["word"]]) == 0xB << (4 * c["nibble"])
-    for c in fx["scales"]:
-        S = np.zeros((N, G), np.float16)
-        S[c["n"], c["g"]] = 1.0
-        _, sc, _ = O.pack(np.zeros((N, K), np.uint8), S, np.zeros((N, G), np.uint8))
-        assert np.nonzero(sc)[0].tolist() == [c["index"]]
-    for c in fx["zeros"]:
-        z = np.zeros((N, G), np.uint8)
-        z[c["n"], c["g"]] = 9
-        _, _, zb = O.pack(np.zeros((N, K), np.uint8), np.zeros((N, G), np.float16), z)
-        assert np.nonzero(zb)[0].tolist() == [c["byte"]]
-        assert int(zb[c["byte"]]) == (9 << 4 if c["high"] else 9)
+    for shp in fx["shapes"]:
+        N, K = shp["N"], shp["K"]
+        G = K // 128
+        words, nsc, nzb = O.packed_sizes(N, K)
+        assert (words, nsc, nzb) == (shp["sizes"]["words"], shp["sizes"]["scales"], shp["sizes"]["zero_bytes"])
+        for c in shp["codes"]:
+            q = np.zeros((N, K), np.uint8)
+            q[c["n"], c["k"]] = 0xB
+            qw, _, _ = O.pack(q, np.zeros((N, G), np.float16), np.zeros((N, G), np.uint8))
+            nz = np.nonzero(qw)[0]
+            assert nz.tolist() == [c["word"]]
+            assert int(qw[c["word"]]) == 0xB << (4 * c["nibble"])
+        for c in shp["scales"]:
+            S = np.zeros((N, G), np.float16)
+            S[c["n"], c["g"]] = 1.0
+            _, sc, _ = O.pack(np.zeros((N, K), np.uint8), S, np.zeros((N, G), np.uint8))
+            assert np.nonzero(sc)[0].tolist() == [c["index"]]
+        for c in shp["zeros"]:
+            z = np.zeros((N, G), np.uint8)
+            z[c["n"], c["g"]] = 9
+            _, _, zb = O.pack(np.zeros((N, K), np.uint8), np.zeros((N, G), np.float16), z)
+            assert np.nonzero(zb)[0].tolist() == [c["byte"]]
+            assert int(zb[c["byte"]]) == (9 << 4 if c["high"] else 9)
 
 
-@pytest.mark.parametrize("N,K", [(128, 128), (300, 256), (16, 384), (513, 640)])
+@pytest.mark.parametrize("N,K", [(128, 128), (300, 256), (16, 384), (513, 640), (7, 1152)])
 def test_layout_roundtrip(N, K):
     rng = np.random.default_rng(N * 31 + K)
     G = K // 128
@@ -324,28 +325,48 @@ def test_layout_roundtrip(N, K):
     q2, S2, z2 = O.unpack(qw, sc, zb, N, K)
     assert np.array_equal(q, q2) and np.array_equal(S.view(np.uint16), S2.view(np.uint16))
     assert np.array_equal(z, z2)
-    # padding rows decode as zeros
+    # padding rows and padding groups decode as zeros
     Np = O.padded_rows(N)
-    qa, Sa, za = O.unpack(qw, sc, zb, Np, K)
-    assert not qa[N:].any() and not Sa[N:].astype(np.float32).any() and not za[N:].any()
+    NT, _, G2, KTp = O.layout_dims(N, K)
+    qa, Sa, za = O.unpack(qw, sc, zb, Np, 128 * 2 * G2)
+    assert not qa[N:].any() and not qa[:, K:].any()
+    assert not Sa[N:].astype(np.float32).any() and not Sa[:, G:].astype(np.float32).any()
+    assert not za[N:].any() and not za[:, G:].any()
 
 
 def test_layout_lane_chunk_holds_its_fragment():
-    """A lane's 16 bytes (4 words) hold rows r, r+8 and k in [16t, 16t+16) of one 16x64 tile."""
-    N, K = 128, 128
-    G = 1
-    n_idx, k_idx = np.meshgrid(np.arange(N), np.arange(K), indexing="ij")
-    for (nt, r, t, kt) in [(0, 0, 0, 0), (3, 5, 2, 1), (7, 7, 3, 1)]:
+    """A lane's 16 bytes (4 words) hold rows r, r+8 and k in [16t, 16t+16) of one 16x64 tile, and a tile's
+    64-k tiles follow one another in memory."""
+    N, K = 128, 256
+    G = 2
+    for (T, r, t, kt) in [(0, 0, 0, 0), (3, 5, 2, 1), (7, 7, 3, 3)]:
         mark = np.zeros((N, K), np.uint8)
-        rows = [nt * 16 + r, nt * 16 + r + 8]
+        rows = [T * 16 + r, T * 16 + r + 8]
         cols = slice(kt * 64 + 16 * t, kt * 64 + 16 * t + 16)
         mark[rows[0], cols] = 1
         mark[rows[1], cols] = 1
         qw, _, _ = O.pack(mark * 15, np.zeros((N, G), np.float16), np.zeros((N, G), np.uint8))
         lane = 4 * r + t
-        base = (kt * 8 + nt) * 128 + lane * 4
+        base = (T * 4 + kt) * 128 + lane * 4
         assert np.nonzero(qw)[0].tolist() == [base, base + 1, base + 2, base + 3]
         assert all(int(w) == 0xFFFFFFFF for w in qw[base:base + 4])
+
+
+def test_layout_tile_streams_are_contiguous():
+    """Everything of tile T (codes, scales, zeros) lies in one contiguous range of each array, in k order."""
+    N, K = 64, 512
+    NT, G, G2, KTp = O.layout_dims(N, K)
+    for T in range(NT):
+        q = np.zeros((N, K), np.uint8)
+        q[16 * T:16 * T + 16] = 15
+        S = np.zeros((N, G), np.float16)
+        S[16 * T:16 * T + 16] = 1.0
+        z = np.zeros((N, G), np.uint8)
+        z[16 * T:16 * T + 16] = 15
+        qw, sc, zb = O.pack(q, S, z)
+        assert np.nonzero(qw)[0].tolist() == list(range(T * KTp * 128, (T + 1) * KTp * 128))
+        assert np.nonzero(sc)[0].tolist() == list(range(T * 2 * G2 * 16, (T + 1) * 2 * G2 * 16))
+        assert np.nonzero(zb)[0].tolist() == list(range(T * 2 * G2 * 8, (T + 1) * 2 * G2 * 8))
 
 
 # ----------------------------------------------------------------------------
@@ -380,3 +401,53 @@ def test_reference_forward_tiny_workload_shapes():
     r = O.reference_forward(x, W)
     assert r["q"].shape == (512, 512) and r["S"].shape == (512, 4) and r["y"].shape == (1, 512)
     assert workloads.n_outlier_channels(512) == 5
+
+
+# ----------------------------------------------------------------------------
+# AWQ scale search
+# ----------------------------------------------------------------------------
+def _search_case_known_optimum(seed=5, M=8, N=32, K=256):
+    """Calibration rows and weights for which alpha = 0.5 quantizes losslessly by construction.
+
+    Channel j has mean |x_j| = 4^k_j (rows are +-4^k_j), so at alpha = 0.5 the scale is s_j = 2^k_j
+    exactly and x' = x / s is exact. The weights are W_nj = m_nj 2^(-6 - k_j) with integer
+    m_nj in 0..15 and every group holding a 0 and a 15, so W s = m 2^-6 sits exactly on the 4-bit grid
+    (lo = 0, S = 2^-6, z = 0) and dequantizes to itself: the output error is exactly zero. Other
+    exponents give non-power-of-two scales, off-grid folded weights and a positive error.
+    """
+    rng = np.random.default_rng(seed)
+    k = np.array([-1, 0, 1, 2] * (K // 4))
+    x = (np.where(rng.random((M, K)) < 0.5, -1.0, 1.0) * (4.0 ** k)[None, :]).astype(np.float16)
+    m = rng.integers(0, 16, (N, K))
+    m[:, 0::128] = 0
+    m[:, 1::128] = 15
+    W = (m * 2.0 ** (-6 - k)[None, :]).astype(np.float16)
+    assert np.array_equal(W.astype(np.float64), m * 2.0 ** (-6 - k)[None, :])   # exact in fp16
+    return x, W
+
+
+def test_search_finds_the_constructed_optimum():
+    x, W = _search_case_known_optimum()
+    alpha, s, errs = O.search_alpha(x, W)
+    assert alpha == 0.5
+    assert np.array_equal(s, (2.0 ** np.array([-1, 0, 1, 2] * 64)).astype(np.float32))
+    assert errs[10] == 0.0
+    assert (np.delete(errs, 10) > 0).all()
+
+
+def test_search_errors_definition_pieces():
+    """The error at alpha = 0 is the plain quantization error of W (no fold: s = mean|x|^0 = 1 and
+    x' = x), written here from the pieces, not from search_errors."""
+    x, W = workloads.random_case(7, 4, 24, 256)
+    errs = O.search_errors(x, W, np.array([0.0], np.float32))
+    q, S, z = O.quantize_groups(W)
+    w_hat = (q.astype(np.float64).reshape(24, 2, 128) - z[..., None]) * S.astype(np.float64)[..., None]
+    y_q = x.astype(np.float64) @ w_hat.reshape(24, 256).T
+    y = x.astype(np.float64) @ W.astype(np.float64).T
+    assert abs(errs[0] - np.sum((y - y_q) ** 2)) <= 1e-12 * np.sum(y ** 2)
+
+
+def test_alpha_grid_is_even_over_unit_interval():
+    g = O.alpha_grid(20)
+    assert g.dtype == np.float32 and g[0] == 0.0 and g[10] == 0.5 and len(g) == 20 and g[-1] < 1.0
+    assert np.allclose(np.diff(g.astype(np.float64)), 0.05)

@@ -129,18 +129,90 @@ def _ptr(t) -> _VP:
     return _VP(t.data_ptr()) if t is not None else _VP(0)
 
 
-def _need(t, dtype, name, dims=None):
+def _need(t, dtype, name, dims=None, require_cuda=True):
     torch = _torch()
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if require_cuda:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.device.index != torch.cuda.current_device():
+            raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                             f"cuda:{torch.cuda.current_device()} (the library runs on the current device)")
     if t.dtype != dtype:
         raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dims is not None and t.dim() != dims:
         raise ValueError(f"{name} must have {dims} dimensions")
+
+
+def _packed_sizes_host(N: int, K: int) -> Tuple[int, int, int]:
+    """Byte sizes of packed layout v2 computed here (used before a library call, so that a caller's
+    buffers are checked against the same figures the library states)."""
+    if N < 1 or K < GROUP_SIZE or K % GROUP_SIZE:
+        return 0, 0, 0
+    tiles, pairs = -(-N // 16), -(-(K // GROUP_SIZE) // 2)
+    return tiles * pairs * 2048, tiles * pairs * 64, tiles * pairs * 16
+
+
+def _check_packed(qweight, scales, zeros, N: int, K: int, require_cuda=True):
+    torch = _torch()
+    _need(qweight, torch.int32, "qweight", require_cuda=require_cuda)
+    _need(scales, torch.float16, "scales", require_cuda=require_cuda)
+    _need(zeros, torch.uint8, "zeros", require_cuda=require_cuda)
+    qb, sb, zb = _packed_sizes_host(N, K)
+    if qb == 0:
+        raise ValueError("N >= 1 and K a positive multiple of 128 are required")
+    if qweight.numel() * 4 < qb or scales.numel() * 2 < sb or zeros.numel() < zb:
+        raise ValueError(f"packed weight tensors are too small for N={N}, K={K}: need {qb}, {sb}, {zb} bytes")
+
+
+def _check_vec(v, K: int, name: str, require_cuda=True):
+    torch = _torch()
+    _need(v, torch.float32, name, 1, require_cuda=require_cuda)
+    if v.numel() != K:
+        raise ValueError(f"{name} must have K={K} elements, got {v.numel()}")
+
+
+def validate_activation_scale(x, s_out, x_scaled, require_cuda=True):
+    torch = _torch()
+    _need(x, torch.float16, "x", 2, require_cuda=require_cuda)
+    M, K = x.shape
+    _check_vec(s_out, K, "s_out", require_cuda)
+    if x_scaled is not None:
+        _need(x_scaled, torch.float16, "x_scaled", 2, require_cuda=require_cuda)
+        if tuple(x_scaled.shape) != (M, K):
+            raise ValueError(f"x_scaled must have shape {(M, K)}, got {tuple(x_scaled.shape)}")
+
+
+def validate_scale_activations(x, s, x_scaled, require_cuda=True):
+    torch = _torch()
+    _need(x, torch.float16, "x", 2, require_cuda=require_cuda)
+    M, K = x.shape
+    _check_vec(s, K, "s", require_cuda)
+    _need(x_scaled, torch.float16, "x_scaled", 2, require_cuda=require_cuda)
+    if tuple(x_scaled.shape) != (M, K):
+        raise ValueError(f"x_scaled must have shape {(M, K)}, got {tuple(x_scaled.shape)}")
+
+
+def validate_quantize(W, fold_scale, out, require_cuda=True):
+    torch = _torch()
+    _need(W, torch.float16, "W", 2, require_cuda=require_cuda)
+    N, K = W.shape
+    if fold_scale is not None:
+        _check_vec(fold_scale, K, "fold_scale", require_cuda)
+    _check_packed(*out, N, K, require_cuda=require_cuda)
+
+
+def validate_linear(x, qweight, scales, zeros, N: int, y, require_cuda=True):
+    torch = _torch()
+    _need(x, torch.float16, "x", 2, require_cuda=require_cuda)
+    M, K = x.shape
+    _check_packed(qweight, scales, zeros, N, K, require_cuda=require_cuda)
+    _need(y, torch.float16, "y", 2, require_cuda=require_cuda)
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"y must have shape {(M, N)}, got {tuple(y.shape)}")
 
 
 def awq_activation_scale(x, alpha: float = 0.5, s_out=None, x_scaled=None, want_scaled: bool = True):
@@ -150,11 +222,9 @@ def awq_activation_scale(x, alpha: float = 0.5, s_out=None, x_scaled=None, want_
     M, K = x.shape
     if s_out is None:
         s_out = torch.empty(K, dtype=torch.float32, device=x.device)
-    _need(s_out, torch.float32, "s_out", 1)
     if want_scaled and x_scaled is None:
         x_scaled = torch.empty_like(x)
-    if x_scaled is not None:
-        _need(x_scaled, torch.float16, "x_scaled", 2)
+    validate_activation_scale(x, s_out, x_scaled)
     st = load_library().awq_activation_scale(_ptr(x), M, K, float(alpha), _ptr(s_out), _ptr(x_scaled),
                                              _stream_ptr())
     _check("awq_activation_scale", st)
@@ -173,16 +243,13 @@ def alloc_packed(N: int, K: int, device="cuda"):
 
 
 def awq_quantize_g128(W, fold_scale=None, out=None):
-    """a2: fold s into W[N,K] and quantize to packed layout v1. Returns (qweight, scales, zeros)."""
+    """a2: fold s into W[N,K] and quantize to packed layout v2. Returns (qweight, scales, zeros)."""
     torch = _torch()
     _need(W, torch.float16, "W", 2)
     N, K = W.shape
-    if fold_scale is not None:
-        _need(fold_scale, torch.float32, "fold_scale", 1)
-    qweight, scales, zeros = out if out is not None else alloc_packed(N, K, W.device)
-    _need(qweight, torch.int32, "qweight")
-    _need(scales, torch.float16, "scales")
-    _need(zeros, torch.uint8, "zeros")
+    out = out if out is not None else alloc_packed(N, K, W.device)
+    validate_quantize(W, fold_scale, out)
+    qweight, scales, zeros = out
     st = load_library().awq_quantize_g128(_ptr(W), _ptr(fold_scale), N, K, _ptr(qweight), _ptr(scales),
                                           _ptr(zeros), _stream_ptr())
     _check("awq_quantize_g128", st)
@@ -192,18 +259,10 @@ def awq_quantize_g128(W, fold_scale=None, out=None):
 def _linear(fn_name: str, x, qweight, scales, zeros, N: int, y=None):
     torch = _torch()
     _need(x, torch.float16, "x", 2)
-    _need(qweight, torch.int32, "qweight")
-    _need(scales, torch.float16, "scales")
-    _need(zeros, torch.uint8, "zeros")
     M, K = x.shape
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=x.device)
-    _need(y, torch.float16, "y", 2)
-    if tuple(y.shape) != (M, N):
-        raise ValueError("y must have shape (M, N)")
-    qb, sb, zb = packed_nbytes(N, K)
-    if qweight.numel() * 4 < qb or scales.numel() * 2 < sb or zeros.numel() < zb:
-        raise ValueError("packed weight tensors are too small for (N, K)")
+    validate_linear(x, qweight, scales, zeros, N, y)
     st = getattr(load_library(), fn_name)(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(y), M, N, K,
                                           _stream_ptr())
     _check(fn_name, st)
@@ -221,7 +280,7 @@ def awq_w4a16_gemm(x, qweight, scales, zeros, N: int, y=None):
 
 
 def awq_w4a16_linear(x, qweight, scales, zeros, N: int, y=None):
-    """gemv for M <= 32, gemm otherwise."""
+    """The decode kernel for small M, the prefill kernel otherwise (the library picks)."""
     return _linear("awq_w4a16_linear", x, qweight, scales, zeros, N, y)
 
 
@@ -266,11 +325,10 @@ def awq_scale_activations(x, s, x_scaled=None):
     """a1 with a stored s: x' = fp16(x / s) (the activation half of the equivalent transform)."""
     torch = _torch()
     _need(x, torch.float16, "x", 2)
-    _need(s, torch.float32, "s", 1)
     M, K = x.shape
     if x_scaled is None:
         x_scaled = torch.empty_like(x)
-    _need(x_scaled, torch.float16, "x_scaled", 2)
+    validate_scale_activations(x, s, x_scaled)
     st = load_library().awq_scale_activations(_ptr(x), _ptr(s), M, K, _ptr(x_scaled), _stream_ptr())
     _check("awq_scale_activations", st)
     return x_scaled

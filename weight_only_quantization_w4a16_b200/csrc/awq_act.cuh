@@ -31,7 +31,7 @@ __device__ __forceinline__ uint64_t f16_abs_units(uint32_t bits) {
   return e == 0 ? static_cast<uint64_t>(m) : (static_cast<uint64_t>(m | 0x400u) << (e - 1));
 }
 
-__global__ void __launch_bounds__(kActThreads) act_scale_kernel(const __half* __restrict__ x, int M, int K,
+__global__ void __launch_bounds__(kActThreads) awq_act_scale_kernel(const __half* __restrict__ x, int M, int K,
                                                                float alpha, float* __restrict__ s_out,
                                                                __half* __restrict__ x_scaled) {
   namespace cg = cooperative_groups;
@@ -141,9 +141,9 @@ __global__ void __launch_bounds__(kActThreads) act_scale_kernel(const __half* __
 }
 
 // Small M (decode): one thread per column, no cluster. The same exact integer column sum,
-// the same float64 statistic and the same fp32 division as act_scale_kernel.
+// the same float64 statistic and the same fp32 division as awq_act_scale_kernel.
 constexpr int kActSmallMaxM = 32;
-__global__ void __launch_bounds__(128) act_scale_small_kernel(const __half* __restrict__ x, int M, int K,
+__global__ void __launch_bounds__(128) awq_act_scale_small_kernel(const __half* __restrict__ x, int M, int K,
                                                              float alpha, float* __restrict__ s_out,
                                                              __half* __restrict__ x_scaled) {
   pdl_enter();
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(128) act_scale_small_kernel(const __half* __re
 
 // x'[m, k] = fp16_rn(fp32(x[m, k]) / s[k]) with a given s (the activation half of the
 // equivalent transform at inference time, s fixed by calibration). One thread per 8 values.
-__global__ void __launch_bounds__(256) scale_activations_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(256) awq_scale_activations_kernel(const __half* __restrict__ x,
                                                                const float* __restrict__ s, long long total8, int K,
                                                                __half* __restrict__ xs) {
   pdl_enter();

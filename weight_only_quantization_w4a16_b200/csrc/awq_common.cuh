@@ -15,7 +15,8 @@
 namespace awq {
 
 // ---------------------------------------------------------------------------
-// Packed layout v1 constants (see include/awq_w4a16.h).
+// Packed layout v2 constants (see include/awq_w4a16.h): 16-row tiles, each tile's codes, scales
+// and zeros contiguous along K in group pairs (2048 + 64 + 16 bytes per tile and pair).
 // ---------------------------------------------------------------------------
 constexpr int kGroup = 128;        // quantization group along K
 constexpr int kKTile = 64;         // k per packed tile
@@ -23,8 +24,13 @@ constexpr int kSuperRows = 128;    // rows per super-tile
 constexpr int kTileRows = 16;      // rows per mma tile
 constexpr int kChunkWords = 128;   // words of one (16-row, 64-k) tile = 512 bytes
 constexpr int kSuperChunkWords = 8 * kChunkWords;  // (128-row, 64-k) = 4096 bytes
+constexpr int kPairCodeBytes = 2048;   // codes of one (tile, group pair)
+constexpr int kPairScaleBytes = 64;    // scales of one (tile, group pair)
+constexpr int kPairZeroBytes = 16;     // zeros of one (tile, group pair)
 
-__host__ __device__ inline int padded_rows(int N) { return (N + kSuperRows - 1) / kSuperRows * kSuperRows; }
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+// Rows rounded up to whole 128-row super-tiles (the prefill kernel's and the quantizer's row blocks).
+__host__ __device__ inline int padded_rows(int N) { return ceil_div(N, kSuperRows) * kSuperRows; }
 
 // ---------------------------------------------------------------------------
 // Device status word and the wait budget for bounded spin-waits.
@@ -144,6 +150,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* m
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst_smem)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -226,8 +240,10 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 // ---------------------------------------------------------------------------
 // Legacy warp-level MMA (register operands), used by the decode kernel.
 // ---------------------------------------------------------------------------
+// A pure register-to-register operation: not volatile, so the compiler may interleave independent
+// accumulator chains.
 __device__ __forceinline__ void mma_m16n8k16_f32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -247,6 +263,23 @@ __device__ __forceinline__ uint32_t lop_or(uint32_t q, uint32_t mask, uint32_t b
   // r = (q & mask) | bits in one LOP3 (immediate LUT 0xEA = (a & b) | c)
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(q), "r"(mask), "r"(bits));
   return r;
+}
+
+// fp16 pair -> two fp32 values through the mixed-precision add f32(h) + (-0.0) (an FMA-pipe
+// instruction; exact for every fp16 value, signed zeros and non-finite values included).
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t v) {
+  float a, b;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %3;\n\tadd.rn.f32.f16 %1, h, %3;\n\t}"
+      : "=f"(a), "=f"(b)
+      : "r"(v), "f"(-0.0f));
+  return make_float2(a, b);
+}
+
+// A small non-negative integer v < 2^23 as fp32 without the conversion unit: the bits of 2^23 + v
+// minus 2^23 (exact).
+__device__ __forceinline__ float small_uint_to_float(uint32_t v) {
+  return __int_as_float(0x4B000000 | v) - 8388608.0f;
 }
 
 __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {

@@ -8,10 +8,12 @@
 // 128-row A operand (one 128-row super-tile of the packed layout), and a
 // tile of BT tokens of x' is the B operand, so every dequantized weight feeds
 // BT tokens. Per CTA (persistent, one per SM):
-//   warp NDQ+4 (one lane): producer — 1-D bulk copies of the packed codes
-//       (4 KB), scales (256 B) and zeros (64 B) of a (super-tile, 64-k) block
-//       and a 2-D TMA load of the x' tile (BT x 64, 128-byte swizzle) into a
-//       STAGES-deep shared-memory ring (mbarrier transaction counts);
+//   warp NDQ+4 (one lane): producer — 3-D TMA boxes of the packed codes
+//       (8 tiles x one 64-k tile = 4 KB), scales (8 x 32 B) and zeros
+//       (8 x 16 B) of a (super-tile, 64-k) block of packed layout v2, and a
+//       2-D TMA load of the x' tile (BT x 64, 128-byte swizzle) into a
+//       STAGES-deep shared-memory ring (mbarrier transaction counts; tiles
+//       past the last one read as zeros);
 //   warps 0..NDQ-1: dequantize codes to fp16 (q - z) * S straight into the
 //       A tile in the canonical K-major 128-byte-swizzle layout (bank-conflict
 //       free 8-byte stores), then fence.proxy.async and arrive;
@@ -42,7 +44,7 @@ struct GemmCfg {
   static constexpr int kB = BT * kKTile * 2;                // x' tile
   static constexpr int kRawQ = kSuperChunkWords * 4;        // 4096 B
   static constexpr int kRawS = 8 * 16 * 2;                  // 256 B
-  static constexpr int kRawZ = 8 * 8;                       // 64 B
+  static constexpr int kRawZ = 8 * 16;                      // 128 B: zeros of the group pair, 8 tiles
   static constexpr int kTx = kB + kRawQ + kRawS + kRawZ;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kA;
@@ -70,9 +72,9 @@ struct GemmCfg {
 
 template <int BT, int STAGES, int NDQ, int CPS>
 __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t* __restrict__ qweight,
-                const __half* __restrict__ scales, const uint8_t* __restrict__ zeros, __half* __restrict__ y, int M,
-                int N, int K) {
+    awq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
+                    __half* __restrict__ y, int M, int N, int K) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,7 +93,6 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   const int MTT = (M + BT - 1) / BT;
   const int ntiles = NST * MTT;
   const int KB = K / kKTile;
-  const int G = K / kGroup;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -107,7 +108,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     *s_abort = 0;
     mbar_fence_init();
   }
-  if (warp == C::kWarpProd && lane == 0) tma_prefetch_desc(&tmap_x);
+  if (warp == C::kWarpProd && lane == 0) {
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_s);
+    tma_prefetch_desc(&tmap_z);
+  }
   if (warp == C::kWarpMma) {
     tmem_alloc(s_tmem, C::kTmemCols);
     tmem_relinquish();
@@ -128,18 +134,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const int st = tile % NST, mt = tile / NST;
-        const uint32_t* qsrc = qweight + static_cast<size_t>(st) * KB * kSuperChunkWords;
-        const __half* ssrc = scales + static_cast<size_t>(st) * G * 128;
-        const uint8_t* zsrc = zeros + static_cast<size_t>(st) * G * 64;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::kTx);
-          bulk_g2s(smem + C::kOffQ + stage * C::kRawQ, qsrc + static_cast<size_t>(kb) * kSuperChunkWords, C::kRawQ,
-                   &full[stage]);
-          bulk_g2s(smem + C::kOffS + stage * C::kRawS, ssrc + static_cast<size_t>(kb >> 1) * 128, C::kRawS,
-                   &full[stage]);
-          bulk_g2s(smem + C::kOffZ + stage * C::kRawZ, zsrc + static_cast<size_t>(kb >> 1) * 64, C::kRawZ,
-                   &full[stage]);
+          tma_load_3d(smem + C::kOffQ + stage * C::kRawQ, &tmap_q, 0, kb, 8 * st, &full[stage]);
+          tma_load_3d(smem + C::kOffS + stage * C::kRawS, &tmap_s, 0, kb >> 1, 8 * st, &full[stage]);
+          tma_load_3d(smem + C::kOffZ + stage * C::kRawZ, &tmap_z, 0, kb >> 2, 8 * st, &full[stage]);
           tma_load_2d(smem + C::kOffB + stage * C::kB, &tmap_x, kb * kKTile, mt * BT, &full[stage]);
           issued_mask |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
           const int nt = c >> 5, lw = c & 31, r = lw >> 2, t = lw & 3;
           const uint4 words = *reinterpret_cast<const uint4*>(rq + nt * kChunkWords + lw * 4);
           const uint32_t sp = rs[nt * 8 + r];                        // (S_r, S_{r+8})
-          const uint32_t zb = rz[nt * 8 + r];
+          const uint32_t zb = rz[nt * 16 + ((kb >> 1) & 1) * 8 + r];
           const uint32_t s_r = __byte_perm(sp, 0, 0x1010);          // (S_r, S_r)
           const uint32_t s_r8 = __byte_perm(sp, 0, 0x3232);         // (S_{r+8}, S_{r+8})
           const uint32_t za = 0x64006400u | ((zb & 0xFu) * 0x00010001u);

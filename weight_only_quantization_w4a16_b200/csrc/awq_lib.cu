@@ -104,12 +104,55 @@ awq_status_t make_x_map(CUtensorMap* map, const void* x, int M, int K, int BT) {
   return r == CUDA_SUCCESS ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
+// The packed arrays of layout v2 as 3-D tensors for the prefill kernel's producer; a box is
+// 8 tiles (one super-tile) of one 64-k tile (codes), one group (scales) or one group pair
+// (zeros), so it lands in shared memory as [tile][...] exactly like a 128-row block.
+//   codes  uint32 {128 words, KTp k-tiles, ntiles}  box {128, 1, 8}
+//   scales uint16 {16, 2*G2 groups, ntiles}         box {16, 1, 8}
+//   zeros  uint8  {16, G2 pairs, ntiles}            box {16, 1, 8}
+awq_status_t make_weight_maps(CUtensorMap* qm, CUtensorMap* sm, CUtensorMap* zm, const void* qw, const void* sc,
+                              const void* zr, int N, int K) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return AWQ_ERR_CUDA;
+  const cuuint64_t nt = static_cast<cuuint64_t>(ceil_div(N, kTileRows));
+  const cuuint64_t g2 = static_cast<cuuint64_t>(ceil_div(K / kGroup, 2));
+  const cuuint32_t estr[3] = {1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {128, 4 * g2, nt};
+    const cuuint64_t strides[2] = {512, 4 * g2 * 512};
+    const cuuint32_t box[3] = {128, 1, 8};
+    if (enc(qm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(qw), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {16, 2 * g2, nt};
+    const cuuint64_t strides[2] = {32, 2 * g2 * 32};
+    const cuuint32_t box[3] = {16, 1, 8};
+    if (enc(sm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(sc), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {16, g2, nt};
+    const cuuint64_t strides[2] = {16, g2 * 16};
+    const cuuint32_t box[3] = {16, 1, 8};
+    if (enc(zm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(zr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return AWQ_ERR_CUDA;
+  }
+  return AWQ_OK;
+}
+
 // --------------------------------------------------------------------------- launch helper
 // Every kernel is launched with programmatic stream serialization (PDL): it may start while the
 // previous kernel of the stream drains, runs its prologue, and waits (griddepcontrol.wait) before
-// touching global memory. cluster_y > 1 adds a (1, cluster_y, 1) thread-block cluster.
+// touching data a predecessor may write. A cluster shape with x > 0 adds a thread-block cluster.
 template <typename... KArgs, typename... Args>
-awq_status_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_y, size_t smem,
+awq_status_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, dim3 cluster, size_t smem,
                        cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -121,11 +164,11 @@ awq_status_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, int clus
   attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[na].val.programmaticStreamSerializationAllowed = 1;
   ++na;
-  if (cluster_y > 0) {
+  if (cluster.x > 0) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = 1;
-    attr[na].val.clusterDim.y = static_cast<unsigned>(cluster_y);
-    attr[na].val.clusterDim.z = 1;
+    attr[na].val.clusterDim.x = cluster.x;
+    attr[na].val.clusterDim.y = cluster.y;
+    attr[na].val.clusterDim.z = cluster.z;
     ++na;
   }
   cfg.attrs = attr;
@@ -154,13 +197,13 @@ int max_active_clusters(Kernel kernel, int threads, size_t smem, int cl, int dev
       if (cache.e[i].dev == dev && cache.e[i].cl == cl && cache.e[i].smem == smem) return cache.e[i].clusters;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cl, cl, 1);
+  cfg.gridDim = dim3(cl * 64, 1, 1);
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(cl);
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+  attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -174,76 +217,128 @@ int max_active_clusters(Kernel kernel, int threads, size_t smem, int cl, int dev
   return n;
 }
 
-template <int MT, int S, int KS, int CW, bool kSumX = false>
+// x' [M, K] fp16 for the decode kernel as a 3-D tensor {64 k, M tokens, K/64 k-tiles}; a box is
+// {64, M, kt_box}: one stage's k-tiles for every token, laid out [k-tile][token][64 k] in shared
+// memory (128-byte rows; 128-byte swizzle when `swizzle`), zero fill past K.
+awq_status_t make_x_map_decode(CUtensorMap* map, const void* x, int M, int K, int kt_box, bool swizzle) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return AWQ_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kKTile), static_cast<cuuint64_t>(M),
+                              static_cast<cuuint64_t>(K / kKTile)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(kKTile) * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kKTile), static_cast<cuuint32_t>(M),
+                             static_cast<cuuint32_t>(kt_box)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
+
+#ifndef AWQ_GEMV_CL
+#define AWQ_GEMV_CL 2
+#endif
+
+template <int MT, int NT, int CW, int D, int SB, int NACC = 2, bool kSumX = false>
 awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
                              int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using Cfg = GemvCfg<MT, S, KS, CW>;
+  using Cfg = GemvCfg<MT, NT, CW, D, SB>;
   static_assert(!kSumX || MT == 1, "activation sums are taken for tokens 0 and 1 only");
-  auto kernel = gemv_kernel<MT, S, KS, CW, kSumX>;
+  auto kernel = awq_gemv_kernel<MT, NT, CW, D, SB, NACC, kSumX>;
   constexpr int kMaxSmem = 227 * 1024;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
   if (st != AWQ_OK) return st;
+  GemvArgs a = {};
+  a.qweight = reinterpret_cast<const uint8_t*>(qw);
+  a.scales = reinterpret_cast<const uint8_t*>(sc);
+  a.zeros = zr;
+  a.y = y;
+  a.M = M;
+  a.N = N;
+  a.ntiles = ceil_div(N, kTileRows);
+  a.g2 = ceil_div(K / kGroup, 2);
+  a.units = ceil_div(a.ntiles, NT);
+  const bool swz = M > 2;
+  a.x_swizzle = swz ? 1 : 0;
+  a.off_scales = Cfg::kCodes;
+  a.off_zeros = a.off_scales + Cfg::kScales;
+  a.off_x = round_up(a.off_zeros + Cfg::kZeros, swz ? 1024 : 128);
+  a.x_box_bytes = 4 * SB * M * 128;
+  a.stage_bytes = round_up(a.off_x + a.x_box_bytes, swz ? 1024 : 128);
   CUtensorMap map;
-  st = make_x_map(&map, x, M, K, Cfg::kMP);
+  st = make_x_map_decode(&map, x, M, K, 4 * SB, swz);
   if (st != AWQ_OK) return st;
-  const int NST = padded_rows(N) / kSuperRows;
-  const int G = K / kGroup;
-  static ClusterOccCache cache;
-  // For each cluster size (K-split), find the co-resident cluster count C whose per-CTA partial
-  // buffers (ceil(NST / C) super-tiles) still let C clusters fit; cost = rounds x K-slice + a
-  // constant for the final reduction. The stream never synchronises before the end.
-  int best_cl = 0, best_clusters = 0, best_units = 0;
-  double best_cost = 1e300;
-  for (int cl = 1; cl <= 8; cl *= 2) {
-    if (cl > G) break;
-#ifdef AWQ_GEMV_FORCE_CL
-    if (cl != AWQ_GEMV_FORCE_CL) continue;
-#endif
-    int clusters = max_active_clusters(kernel, Cfg::kThreads, Cfg::smem_bytes(M, 1), cl, dev, cache);
-    int units = 0;
-    for (int it = 0; it < 6 && clusters > 0; ++it) {
-      clusters = std::min(clusters, NST);
-      units = (NST + clusters - 1) / clusters;
-      const size_t smem = Cfg::smem_bytes(M, units);
-      if (smem > static_cast<size_t>(kMaxSmem)) { clusters = 0; break; }
-      const int c2 = max_active_clusters(kernel, Cfg::kThreads, smem, cl, dev, cache);
-      if (c2 >= clusters) break;
-      clusters = c2;
+  // clusters: CL CTAs each, about one CTA per SM, never more clusters than units
+  // CL CTAs per cluster, at most 32 workers (warps) per cluster: a unit's contributors then fit
+  // one warp's lanes in the reduction
+  int cl = AWQ_GEMV_CL;
+  while (cl > 1 && (a.units < cl || cl * CW > 32)) cl /= 2;
+  static_assert(CW <= 32, "warps per CTA");
+  int clusters = std::max(1, std::min(num_sms / cl, a.units));
+  // partial-sum records per warp: the most units one warp's item range touches
+  const long long Wc = static_cast<long long>(cl) * CW;
+  int R = 1;
+  for (int c = 0; c < clusters; ++c) {
+    const long long u0 = static_cast<long long>(c) * a.units / clusters;
+    const long long u1 = static_cast<long long>(c + 1) * a.units / clusters;
+    const long long L = (u1 - u0) * a.g2;
+    for (long long w = 0; w < Wc; ++w) {
+      const long long lo = w * L / Wc, hi = (w + 1) * L / Wc;
+      if (hi > lo) R = std::max(R, static_cast<int>((hi - 1) / a.g2 - lo / a.g2 + 1));
     }
-    if (clusters <= 0) continue;
-    const double cost = units * static_cast<double>((G + cl - 1) / cl) + 4.0;
-    if (cost < best_cost) { best_cost = cost; best_cl = cl; best_clusters = clusters; best_units = units; }
   }
-  if (best_cl == 0) return AWQ_ERR_UNSUPPORTED;
-  return launch_ex(kernel, dim3(best_clusters, best_cl, 1), dim3(Cfg::kThreads, 1, 1), best_cl,
-                   Cfg::smem_bytes(M, best_units), stream, map, qw, sc, zr, y, M, N, K, best_units);
+  a.rec_per_warp = R;
+  const size_t smem = static_cast<size_t>(CW) * D * a.stage_bytes +
+                      static_cast<size_t>(CW) * R * NT * kTileRows * M * 4 + static_cast<size_t>(CW) * D * 8 + 16 + 1024;
+  if (smem > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
+  static ClusterOccCache cache;
+  const int fit = max_active_clusters(kernel, Cfg::kThreads, smem, cl, dev, cache);
+  if (fit < 1) return AWQ_ERR_UNSUPPORTED;
+  if (clusters > fit) {
+    // fewer clusters than SMs / CL can be resident at once: use what fits (recompute R)
+    clusters = fit;
+    R = 1;
+    for (int c = 0; c < clusters; ++c) {
+      const long long u0 = static_cast<long long>(c) * a.units / clusters;
+      const long long u1 = static_cast<long long>(c + 1) * a.units / clusters;
+      const long long L = (u1 - u0) * a.g2;
+      for (long long w = 0; w < Wc; ++w) {
+        const long long lo = w * L / Wc, hi = (w + 1) * L / Wc;
+        if (hi > lo) R = std::max(R, static_cast<int>((hi - 1) / a.g2 - lo / a.g2 + 1));
+      }
+    }
+    a.rec_per_warp = R;
+  }
+  a.clusters = clusters;
+  const size_t smem2 = static_cast<size_t>(CW) * D * a.stage_bytes +
+                       static_cast<size_t>(CW) * a.rec_per_warp * NT * kTileRows * M * 4 +
+                       static_cast<size_t>(CW) * D * 8 + 16 + 1024;
+  if (smem2 > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
+  return launch_ex(kernel, dim3(clusters * cl, 1, 1), dim3(Cfg::kThreads, 1, 1), dim3(cl, 1, 1), smem2, stream, map,
+                   a);
 }
 
-// Compile-time tuning of the decode kernel per token tile: stages, 64-k tiles per stage,
-// consumer warps. Measured on the Llama-2-7B and 70B decode shapes: larger stages (fewer
-// barrier round trips per weight) win as long as two CTAs still fit on an SM; 4 consumer
-// warps up to M = 16, 8 above, where the extra warps hide the longer mma chains.
-#ifndef AWQ_GEMV1_STAGES
-#define AWQ_GEMV1_STAGES 2
-#endif
-#ifndef AWQ_GEMV1_KS
-#define AWQ_GEMV1_KS 8
-#endif
+// Compile-time tuning of the decode kernel per token tile: warps per CTA, ring stages per warp,
+// group pairs per stage, accumulator chains, and the M <= 2 form (codes as subnormals, zero
+// point through the activation sums).
 #ifndef AWQ_GEMV1_CW
-#define AWQ_GEMV1_CW 4
+#define AWQ_GEMV1_CW 8
 #endif
-#ifndef AWQ_GEMV2_STAGES
-#define AWQ_GEMV2_STAGES 3
+#ifndef AWQ_GEMV1_D
+#define AWQ_GEMV1_D 2
 #endif
-#ifndef AWQ_GEMV2_KS
-#define AWQ_GEMV2_KS 4
+#ifndef AWQ_GEMV1_SB
+#define AWQ_GEMV1_SB 2
 #endif
-#ifndef AWQ_GEMV4_STAGES
-#define AWQ_GEMV4_STAGES 3
+#ifndef AWQ_GEMV1_NACC
+#define AWQ_GEMV1_NACC 4
 #endif
-#ifndef AWQ_GEMV4_KS
-#define AWQ_GEMV4_KS 4
+#ifndef AWQ_GEMV_SUMX
+#define AWQ_GEMV_SUMX 0
 #endif
 
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
@@ -251,18 +346,14 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
   const int mt = (M + 7) / 8;
   switch (mt) {
     case 1:
-      // M <= 2: codes as fp16 subnormals (one AND per pair) and the zero point through the
-      // activation sums, which the warp takes from the activation box at little cost
-      if (M <= 2)
-        return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, AWQ_GEMV1_CW, true>(x, qw, sc, zr, y, M, N, K, dev,
-                                                                                     num_sms, stream);
-      return launch_gemv_cfg<1, AWQ_GEMV1_STAGES, AWQ_GEMV1_KS, AWQ_GEMV1_CW>(x, qw, sc, zr, y, M, N, K, dev, num_sms,
-                                                                             stream);
-    case 2:
-      return launch_gemv_cfg<2, AWQ_GEMV2_STAGES, AWQ_GEMV2_KS, 4>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 3: return launch_gemv_cfg<3, 3, 4, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    default:
-      return launch_gemv_cfg<4, AWQ_GEMV4_STAGES, AWQ_GEMV4_KS, 8>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      if (AWQ_GEMV_SUMX && M <= 2)
+        return launch_gemv_cfg<1, 1, AWQ_GEMV1_CW, AWQ_GEMV1_D, AWQ_GEMV1_SB, AWQ_GEMV1_NACC, true>(
+            x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      // 3 <= M <= 8: the x' box grows with M, so stages hold one group pair
+      return launch_gemv_cfg<1, 1, 8, 2, 1, AWQ_GEMV1_NACC>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 2: return launch_gemv_cfg<2, 2, 4, 3, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    case 3: return launch_gemv_cfg<3, 2, 4, 2, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    default: return launch_gemv_cfg<4, 2, 4, 2, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
   }
 }
 
@@ -271,17 +362,19 @@ template <int BT, int STAGES, int NDQ, int CPS = 1>
 awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
                              int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS>;
-  auto kernel = gemm_kernel<BT, STAGES, NDQ, CPS>;
+  auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS>;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, C::kSmem, dev, smem_done);
   if (st != AWQ_OK) return st;
-  CUtensorMap map;
-  st = make_x_map(&map, x, M, K, BT);
+  CUtensorMap xmap, qmap, smap, zmap;
+  st = make_x_map(&xmap, x, M, K, BT);
+  if (st != AWQ_OK) return st;
+  st = make_weight_maps(&qmap, &smap, &zmap, qw, sc, zr, N, K);
   if (st != AWQ_OK) return st;
   const long long tiles = static_cast<long long>(padded_rows(N) / kSuperRows) * ((M + BT - 1) / BT);
   const int grid = static_cast<int>(std::min<long long>(tiles, static_cast<long long>(CPS) * num_sms));
-  return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), 0, C::kSmem, stream, map, qw, sc, zr, y, M, N,
-                   K);
+  return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), dim3(0, 0, 0), C::kSmem, stream, xmap, qmap,
+                   smap, zmap, y, M, N, K);
 }
 
 // Compile-time tuning of the prefill kernel: dequantization warps, ring stages per token tile
@@ -329,14 +422,24 @@ awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, 
   }
 }
 
+// Rows are limited so that every count below fits an int: N <= 2^31 - 2^7 and N * K <= 2^34.
+constexpr long long kMaxRows = (1ll << 31) - 128;
+inline bool rows_ok(int N, int K) {
+  return N >= 1 && N <= kMaxRows && static_cast<long long>(ceil_div(N, kTileRows)) * kTileRows * K <= (1ll << 34);
+}
+
 awq_status_t check_linear_args(const void* x, const void* qw, const void* sc, const void* zr, const void* y, int M,
                                int N, int K) {
   if (!x || !qw || !sc || !zr || !y) return AWQ_ERR_INVALID_ARG;
-  if (M < 1 || N < 1 || K < kGroup || K % kGroup != 0) return AWQ_ERR_INVALID_ARG;
-  if (static_cast<long long>(M) * K > (1ll << 31) - 1 || static_cast<long long>(padded_rows(N)) * K > (1ll << 34))
-    return AWQ_ERR_INVALID_ARG;
+  if (M < 1 || K < kGroup || K % kGroup != 0 || !rows_ok(N, K)) return AWQ_ERR_INVALID_ARG;
+  if (static_cast<long long>(M) * K > (1ll << 31) - 1) return AWQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(qw) || !aligned16(sc) || !aligned16(zr) || !aligned16(y)) return AWQ_ERR_MISALIGNED;
   return AWQ_OK;
+}
+
+// Packed sizes of layout v2: per (16-row tile, group pair) 2048 + 64 + 16 bytes.
+inline size_t tile_pairs(int N, int K) {
+  return static_cast<size_t>(ceil_div(N, kTileRows)) * static_cast<size_t>(ceil_div(K / kGroup, 2));
 }
 
 }  // namespace
@@ -346,7 +449,7 @@ using namespace awq;
 
 extern "C" {
 
-int awq_layout_version(void) { return 1; }
+int awq_layout_version(void) { return 2; }
 
 const char* awq_status_string(int status) {
   switch (status) {
@@ -365,16 +468,16 @@ awq_status_t awq_check_config(int bits, int group_size, int zero_point) {
 }
 
 size_t awq_qweight_bytes(int N, int K) {
-  if (N < 1 || K < kGroup || K % kGroup) return 0;
-  return static_cast<size_t>(padded_rows(N)) * K / 2;
+  if (K < kGroup || K % kGroup || !rows_ok(N, K)) return 0;
+  return tile_pairs(N, K) * kPairCodeBytes;
 }
 size_t awq_scales_bytes(int N, int K) {
-  if (N < 1 || K < kGroup || K % kGroup) return 0;
-  return static_cast<size_t>(padded_rows(N)) * (K / kGroup) * 2;
+  if (K < kGroup || K % kGroup || !rows_ok(N, K)) return 0;
+  return tile_pairs(N, K) * kPairScaleBytes;
 }
 size_t awq_zeros_bytes(int N, int K) {
-  if (N < 1 || K < kGroup || K % kGroup) return 0;
-  return static_cast<size_t>(padded_rows(N)) * (K / kGroup) / 2;
+  if (K < kGroup || K % kGroup || !rows_ok(N, K)) return 0;
+  return tile_pairs(N, K) * kPairZeroBytes;
 }
 
 awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha, float* s_out, uint16_t* x_scaled,
@@ -387,13 +490,13 @@ awq_status_t awq_activation_scale(const uint16_t* x, int M, int K, float alpha, 
   awq_status_t st = current_device(&dev, &sms);
   if (st != AWQ_OK) return st;
   if (M <= kActSmallMaxM)
-    return launch_ex(act_scale_small_kernel, dim3((K + 127) / 128, 1, 1), dim3(128, 1, 1), 0, 0,
+    return launch_ex(awq_act_scale_small_kernel, dim3((K + 127) / 128, 1, 1), dim3(128, 1, 1), dim3(0, 0, 0), 0,
                      reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), M, K, alpha, s_out,
                      reinterpret_cast<__half*>(x_scaled));
   int cl = 1;
   while (cl < 8 && cl * 256 < M) cl *= 2;
   const int slabs = (K + kActCols - 1) / kActCols;
-  return launch_ex(act_scale_kernel, dim3(slabs, cl, 1), dim3(kActThreads, 1, 1), cl, 0,
+  return launch_ex(awq_act_scale_kernel, dim3(slabs, cl, 1), dim3(kActThreads, 1, 1), dim3(1, cl, 1), 0,
                         reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), M, K, alpha,
                         s_out, reinterpret_cast<__half*>(x_scaled));
 }
@@ -409,7 +512,8 @@ awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int
   const long long total8 = static_cast<long long>(M) * K / 8;
   const long long blocks = (total8 + 255) / 256;
   if (blocks > 2147483647ll) return AWQ_ERR_INVALID_ARG;
-  return launch_ex(scale_activations_kernel, dim3(static_cast<unsigned>(blocks), 1, 1), dim3(256, 1, 1), 0, 0,
+  return launch_ex(awq_scale_activations_kernel, dim3(static_cast<unsigned>(blocks), 1, 1), dim3(256, 1, 1),
+                   dim3(0, 0, 0), 0,
                    reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const __half*>(x), s, total8, K,
                    reinterpret_cast<__half*>(x_scaled));
 }
@@ -417,8 +521,7 @@ awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int
 awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K, uint32_t* qweight,
                                uint16_t* scales, uint8_t* zeros, awq_stream_t stream) {
   if (!W || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
-  if (N < 1 || K < kGroup || K % kGroup != 0) return AWQ_ERR_INVALID_ARG;
-  if (static_cast<long long>(padded_rows(N)) * K > (1ll << 34)) return AWQ_ERR_INVALID_ARG;
+  if (K < kGroup || K % kGroup != 0 || !rows_ok(N, K)) return AWQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(fold_scale))
     return AWQ_ERR_MISALIGNED;
   int dev, sms;
@@ -439,16 +542,18 @@ awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N
       return AWQ_ERR_CUDA;
   }
   static std::atomic<uint64_t> done_f{0}, done_n{0};
-  st = fold_scale ? ensure_smem(quantize_g128_kernel<true>, kQSmem, dev, done_f)
-                  : ensure_smem(quantize_g128_kernel<false>, kQSmem, dev, done_n);
+  st = fold_scale ? ensure_smem(awq_quantize_g128_kernel<true>, kQSmem, dev, done_f)
+                  : ensure_smem(awq_quantize_g128_kernel<false>, kQSmem, dev, done_n);
   if (st != AWQ_OK) return st;
   const long long units = static_cast<long long>(padded_rows(N) / kSuperRows) * (K / kGroup);
   const int grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(AWQ_QUANT_MINBLOCKS) * sms));
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (fold_scale)
-    return launch_ex(quantize_g128_kernel<true>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), 0, kQSmem, s, map,
+    return launch_ex(awq_quantize_g128_kernel<true>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), dim3(0, 0, 0), kQSmem, s,
+                     map,
                      fold_scale, N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
-  return launch_ex(quantize_g128_kernel<false>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), 0, kQSmem, s, map,
+  return launch_ex(awq_quantize_g128_kernel<false>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), dim3(0, 0, 0), kQSmem, s,
+                   map,
                    static_cast<const float*>(nullptr), N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
 }
 

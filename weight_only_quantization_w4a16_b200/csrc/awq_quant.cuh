@@ -36,7 +36,7 @@
 // (16 rows each) work. Lanes l and l^8 hold the two halves of one row's group
 // (their swizzled 16-byte reads are bank-conflict free); rows r and r+8 live
 // in lanes l and l^16, which trade 4-code quads with one shuffle per word to
-// assemble packed layout v1.
+// assemble packed layout v2.
 #pragma once
 
 #include "awq_common.cuh"
@@ -107,7 +107,7 @@ constexpr int kQThreads = (kQComputeWarps + 1) * 32;        // + 1 producer warp
 constexpr int kQSmem = kQStages * kQStageBytes + 2 * kQStages * 8 + 16 + 1024;
 
 template <bool kFold>
-__global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_kernel(const __grid_constant__ CUtensorMap tmap_w,
+__global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g128_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                  const float* __restrict__ fold, int N, int K,
                                                                  uint32_t* __restrict__ qweight,
                                                                  __half* __restrict__ scales,
@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = K / kGroup;
-  const int KT = K / kKTile;
+  const int G2 = ceil_div(G, 2);
+  const int KTp = 4 * G2;              // k-tiles per tile in packed layout v2 (padded to group pairs)
+  const int ntiles = ceil_div(N, kTileRows);
   const int ST = padded_rows(N) / kSuperRows;
   const int units = ST * G;
   if (threadIdx.x == 0) {
@@ -302,30 +304,42 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) quantize_g128_
 
     // ---- assemble words: lane with h = 0 builds k-tile 2g, lane with h = 1 builds k-tile 2g+1.
     // Chunk i covers k-tile (i >> 2), column block t = (i & 3), steps s = 2*half + sbh.
-    uint32_t* out = qweight + (static_cast<size_t>(st) * KT + 2 * g + h) * kSuperChunkWords +
-                    static_cast<size_t>(nt) * kChunkWords;
+    // Tile T = 8 st + nt of packed layout v2: its k-tiles follow one another (KTp per tile).
+    const int T = st * 8 + nt;
+    if (T < ntiles) {
+      uint32_t* out = qweight + (static_cast<size_t>(T) * KTp + 2 * g + h) * kChunkWords;
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      uint32_t w2[2];
+      for (int t = 0; t < 4; ++t) {
+        uint32_t w2[2];
 #pragma unroll
-      for (int sbh = 0; sbh < 2; ++sbh) {
-        const uint32_t send = h ? quad[t][sbh] : quad[4 + t][sbh];
-        const uint32_t mine = h ? quad[4 + t][sbh] : quad[t][sbh];
-        const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
-        const uint32_t a = h ? recv : mine;   // row r
-        const uint32_t b = h ? mine : recv;   // row r + 8
-        w2[sbh] = __byte_perm(a | (b << 4), 0u, 0x3120);
+        for (int sbh = 0; sbh < 2; ++sbh) {
+          const uint32_t send = h ? quad[t][sbh] : quad[4 + t][sbh];
+          const uint32_t mine = h ? quad[4 + t][sbh] : quad[t][sbh];
+          const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 16);
+          const uint32_t a = h ? recv : mine;   // row r
+          const uint32_t b = h ? mine : recv;   // row r + 8
+          w2[sbh] = __byte_perm(a | (b << 4), 0u, 0x3120);
+        }
+        *reinterpret_cast<uint2*>(out + (4 * r + t) * 4 + 2 * half) = make_uint2(w2[0], w2[1]);
       }
-      *reinterpret_cast<uint2*>(out + (4 * r + t) * 4 + 2 * half) = make_uint2(w2[0], w2[1]);
-    }
-
-    // ---- scales and zero points
-    const size_t meta = (static_cast<size_t>(st) * G + g) * 8 + nt;
-    const int zi = valid ? __float2int_rz(zf) : 0;
-    const int z_hi = __shfl_xor_sync(0xFFFFFFFFu, zi, 16);
-    if (half == 0) {
-      scales[meta * 16 + 2 * r + h] = valid ? S : __ushort_as_half(0);
-      if (h == 0) zeros[meta * 8 + r] = static_cast<uint8_t>(zi | (z_hi << 4));
+      // ---- scales and zero points
+      const size_t meta = static_cast<size_t>(T) * 2 * G2 + g;
+      const int zi = valid ? __float2int_rz(zf) : 0;
+      const int z_hi = __shfl_xor_sync(0xFFFFFFFFu, zi, 16);
+      if (half == 0) {
+        scales[meta * 16 + 2 * r + h] = valid ? S : __ushort_as_half(0);
+        if (h == 0) zeros[meta * 8 + r] = static_cast<uint8_t>(zi | (z_hi << 4));
+      }
+      // an odd group count leaves one padding group per tile: code 0, scale 0, zero 0
+      if ((G & 1) && g == G - 1) {
+        uint32_t* pad = qweight + (static_cast<size_t>(T) * KTp + 2 * G + h) * kChunkWords;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) *reinterpret_cast<uint2*>(pad + (4 * r + t) * 4 + 2 * half) = make_uint2(0u, 0u);
+        if (half == 0) {
+          scales[(meta + 1) * 16 + 2 * r + h] = __ushort_as_half(0);
+          if (h == 0) zeros[(meta + 1) * 8 + r] = 0;
+        }
+      }
     }
   }
   __threadfence();   // this thread's codes, scales and zeros are visible device-wide before it exits
