@@ -16,6 +16,8 @@ Sub-records in the same JSON line, each with its own roofline:
   quantize      the fold + quantizer over each full Llama-2-70B layer, GB/s
   act_scale     the activation statistic + scaling at 4096 x 4096, GB/s
   full_path     one pass of every row of the path (a1 + a2 + a3 per layer) on the default workload
+  decode_layer_chain  one Llama-2-7B block's linear layers at M = 1 as a dependent chain (scaling,
+                fused q/k/v, o_proj, fused gate/up SiLU*up, down) in a CUDA graph
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME] [--m M]
 
@@ -644,6 +646,11 @@ def sub_records(torch, P, timer, dev, l2, hbm_peak, tc_peak, tc_sus, peak_src, w
     ba = bytes_act_scale(4096, 4096)
     out["act_scale"] = {"kernel": "awq_act_scale_kernel", "bound": "hbm", "shape": "M=4096, K=4096", "us": us,
                         "GBps": ba / us / 1e3, "frac": ba / us / 1e3 / hbm_peak, "peak": hbm_peak}
+    # a dependent decode chain of one Llama-2-7B block at M = 1: scale -> fused q/k/v (split) ->
+    # scale -> o_proj -> scale -> fused gate+up (SiLU * up) -> scale -> down, each layer fed by the
+    # previous output (q stands in for the attention output), weights rotated through >= 4x L2
+    if M == 1 and wl.name == "llama2_7b_decode_m1":
+        out["decode_layer_chain"] = decode_layer_chain(torch, P, timer, dev, l2, hbm_peak, wl)
     # one pass of every row of the path on this workload: a1 + a2 + linear per layer (full fp16 W read)
     if M <= 32:
         Ws = [torch.from_numpy(workloads.layer_inputs(wl, i, M)[1]).to(dev) for i in range(len(L))]
@@ -660,6 +667,50 @@ def sub_records(torch, P, timer, dev, l2, hbm_peak, tc_peak, tc_sus, peak_src, w
                             "note": "activation statistic + fold/quantize + decode GEMV for every layer of the "
                                     "workload (fp16 weights re-quantized every step)"}
     return out
+
+
+def decode_layer_chain(torch, P, timer, dev, l2, hbm_peak, wl):
+    """Times the dependent chain of a Llama-2-7B block's linear layers at M = 1 (see sub_records)."""
+    layers = []
+    for li, layer in enumerate(wl.layers):
+        x, W = workloads.layer_inputs(wl, li, 1)
+        with torch.cuda.stream(timer.stream):
+            s, _ = P.awq_activation_scale(torch.from_numpy(x).to(dev), 0.5, want_scaled=False)
+            Wd = torch.from_numpy(W).to(dev)
+            pk = P.awq_quantize_g128(Wd, s)
+            del Wd
+        layers.append({"N": layer.N, "K": layer.K, "s": s, "packed": [pk]})
+    nset = rotation_sets(sum(packed_bytes(d["N"], d["K"]) for d in layers), l2)
+    for d in layers:
+        d["packed"] += [tuple(t.clone() for t in d["packed"][0]) for _ in range(nset - 1)]
+    qkv, o, gu, down = layers
+    x0 = torch.from_numpy(workloads.layer_inputs(wl, 0, 1)[0]).to(dev)
+    xs = torch.empty((1, 11008), dtype=torch.float16, device=dev)
+    q, k, v = (torch.empty((1, 4096), dtype=torch.float16, device=dev) for _ in range(3))
+    yo = torch.empty((1, 4096), dtype=torch.float16, device=dev)
+    h = torch.empty((1, 11008), dtype=torch.float16, device=dev)
+    y = torch.empty((1, 4096), dtype=torch.float16, device=dev)
+
+    def chain(i):
+        c = i % nset
+        P.awq_scale_activations(x0, qkv["s"], xs[:, :4096])
+        P.awq_w4a16_linear_qkv(xs[:, :4096], *qkv["packed"][c], 4096, 4096, out=(q, k, v))
+        P.awq_scale_activations(q, o["s"], xs[:, :4096])
+        P.awq_w4a16_gemv(xs[:, :4096], *o["packed"][c], 4096, yo)
+        P.awq_scale_activations(yo, gu["s"], xs[:, :4096])
+        P.awq_w4a16_linear_silu_mul(xs[:, :4096], *gu["packed"][c], 11008, h)
+        P.awq_scale_activations(h, down["s"], xs)
+        P.awq_w4a16_gemv(xs, *down["packed"][c], 4096, y)
+
+    us, g = per_launch_us(timer, chain, launches=32)
+    del g
+    wbytes = sum(2 * d["N"] * d["K"] for d in layers)
+    alg = sum(bytes_linear(1, d["N"], d["K"]) for d in layers)
+    return {"us_per_step": us, "launches_per_step": 8, "effective_weight_GBps": wbytes / us / 1e3,
+            "GBps": alg / us / 1e3, "frac": alg / us / 1e3 / hbm_peak,
+            "note": "one Llama-2-7B block's linear layers at M = 1 as a dependent chain in a CUDA graph with "
+                    "programmatic dependent launch: scale + fused q/k/v, scale + o_proj, scale + fused "
+                    "gate/up SiLU*up, scale + down; 32 steps back to back over rotated weights"}
 
 
 def end_to_end(torch, P, stream, host, L, M, steps, world, decode):

@@ -177,6 +177,54 @@ AWQ_API awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight
                               const uint8_t* zeros, uint16_t* y, int M, int N, int K,
                               awq_stream_t stream);
 
+/* Fused-module epilogues ("transformers - AWQ" section 3: the attention
+ * projections fused in the order query, key, value, with num_key_value_heads
+ * below num_attention_heads giving narrower keys and values; the MLP layers
+ * fused in the order gate, up, down). Same arguments, layout and weight
+ * prefetch rule as awq_w4a16_linear (the decode kernel for M <= 32, the
+ * prefill kernel above), with the output written differently:
+ *
+ * awq_w4a16_linear_qkv: the weight holds N = Nq + 2*Nkv rows (Nq query rows,
+ *   then Nkv key rows, then Nkv value rows); the output goes to
+ *   yq [M, Nq], yk [M, Nkv], yv [M, Nkv] (fp16, row-major, 16-byte aligned).
+ *   Requires Nq >= 1, Nkv >= 1.
+ *
+ * awq_w4a16_linear_silu_mul: the weight holds N = 2*I rows (I gate rows,
+ *   then I up rows), I a multiple of 16; the output is
+ *   h [M, I] = SiLU(x . Wgate^T) * (x . Wup^T), SiLU(v) = v / (1 + e^-v),
+ *   evaluated in fp32 on the fp32 sums (the pages name the fused MLP of Llama
+ *   and Mistral, whose gate activation is SiLU), fp16 output. */
+AWQ_API awq_status_t awq_w4a16_linear_qkv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                          const uint8_t* zeros, uint16_t* yq, uint16_t* yk, uint16_t* yv,
+                                          int M, int Nq, int Nkv, int K, awq_stream_t stream);
+AWQ_API awq_status_t awq_w4a16_linear_silu_mul(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                               const uint8_t* zeros, uint16_t* h, int M, int I, int K,
+                                               awq_stream_t stream);
+
+/* AWQ scale search (llm-awq README "Usage" step 1: the AWQ search picks the
+ * scales on calibration data; CSDN VPTQ blog "02.02 AWQ": scales from offline
+ * activation statistics, no backpropagation). For each candidate exponent
+ * alpha_i the whole path runs on the calibration rows:
+ *   s = max(mean_m |x_mk|, 1e-8)^alpha_i, x' = fp16(x / s), codes of fold(W, s),
+ *   y_i = x' . dequant^T (fp16, the decode or prefill kernel by M),
+ *   err[i] = sum_{m,n} (y_ref[m,n] - y_i[m,n])^2 in float64,
+ * with y_ref = x . W^T (fp16 inputs, fp32 accumulation) computed once.
+ *   x       fp16 [M, K] calibration rows (device);  W fp16 [N, K] (device)
+ *   alphas  float [n_alpha] HOST array of candidates (finite), 1 <= n_alpha <= 4096
+ *   err     double [n_alpha] (device, 8-byte aligned): the squared errors
+ *   best    int [1] (device): index of the first smallest err
+ *   workspace (device, 16-byte aligned) of at least
+ *           awq_search_workspace_bytes(M, N, K) bytes; the library allocates nothing.
+ * The workspace holds y_ref, y_i, s, x', the packed weights of the candidate
+ * being scored and the error reduction's partial sums; its contents after the
+ * call are those of the last candidate. Errors are reproducible from call to
+ * call (fixed reduction order). Requires 1 <= M <= 1048560, K >= 128,
+ * K % 128 == 0, M*N and M*K < 2^31. */
+AWQ_API size_t awq_search_workspace_bytes(int M, int N, int K);
+AWQ_API awq_status_t awq_search_alpha(const uint16_t* x, const uint16_t* W, int M, int N, int K,
+                                      const float* alphas, int n_alpha, double* err, int* best,
+                                      void* workspace, size_t workspace_bytes, awq_stream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word of the
  * current device. Returns AWQ_ERR_TIMEOUT if a kernel since the last poll gave
  * up a bounded wait (its outputs are then undefined), AWQ_ERR_CUDA if the

@@ -201,6 +201,35 @@ def check_tolerance(y: np.ndarray, y_ref: np.ndarray, rel_fro: float = 2e-3, max
 
 
 # --------------------------------------------------------------------------
+# Fused epilogues of the fused-N layers ("transformers - AWQ" section 3)
+# --------------------------------------------------------------------------
+def silu(v: np.ndarray) -> np.ndarray:
+    """SiLU(v) = v / (1 + exp(-v)) in float64 (the Llama/Mistral MLP activation)."""
+    v = np.asarray(v, np.float64)
+    return v / (1.0 + np.exp(-v))
+
+
+def gate_up_silu(y_gate_up: np.ndarray) -> np.ndarray:
+    """h[M, I] = SiLU(y[:, :I]) * y[:, I:] for the fused gate+up output y[M, 2I] (gate rows first).
+
+    [HF-AWQ] section 3: the fused MLP module takes the gate, up and down layers in that order;
+    the gate/up pair of Llama and Mistral (the architectures the section names) combine as
+    SiLU(gate) * up before the down projection. The pages print no activation; reading: SiLU.
+    """
+    y = np.asarray(y_gate_up, np.float64)
+    I = y.shape[1] // 2
+    return silu(y[:, :I]) * y[:, I:]
+
+
+def split_qkv(y_qkv: np.ndarray, n_q: int, n_kv: int):
+    """(q, k, v) = the column blocks [0, n_q), [n_q, n_q + n_kv), [n_q + n_kv, n_q + 2 n_kv) of the
+    fused q/k/v output ([HF-AWQ] section 3: attention layers fused in the order query, key, value;
+    num_key_value_heads < num_attention_heads gives the narrower k and v of grouped-query attention)."""
+    y = np.asarray(y_qkv)
+    return y[:, :n_q], y[:, n_q:n_q + n_kv], y[:, n_q + n_kv:n_q + 2 * n_kv]
+
+
+# --------------------------------------------------------------------------
 # AWQ scale search (the exponent alpha of the activation statistic)
 # --------------------------------------------------------------------------
 def alpha_grid(n_grid: int = 20) -> np.ndarray:

@@ -33,7 +33,8 @@ def _declared():
 def test_header_declares_the_path():
     names = _declared()
     for n in ["awq_activation_scale", "awq_scale_activations", "awq_quantize_g128", "awq_w4a16_gemv",
-              "awq_w4a16_gemm", "awq_w4a16_linear", "awq_poll_device_status", "awq_layout_version"]:
+              "awq_w4a16_gemm", "awq_w4a16_linear", "awq_poll_device_status", "awq_layout_version",
+              "awq_search_alpha", "awq_search_workspace_bytes"]:
         assert n in names
 
 
@@ -106,6 +107,23 @@ def test_argument_checks_fail_before_any_device_call(lib):
     assert lib.awq_w4a16_gemm(V(A), V(A), V(A), V(A), V(A), 64, 2147483600, 128, None) == 1
     assert lib.awq_quantize_g128(V(A), None, 2147483647, 128, V(A), V(A), V(A), None) == 1
     assert lib.awq_w4a16_linear(V(A), V(A), V(A), V(A), V(A), 1, 2 ** 27, 256, None) == 1
+    # the scale search: bad shapes, null outputs, a short workspace, a non-finite candidate
+    a1 = (ctypes.c_float * 1)(0.5)
+    anan = (ctypes.c_float * 1)(float("nan"))
+    assert lib.awq_search_workspace_bytes(0, 16, 128) == 0 and lib.awq_search_workspace_bytes(4, 16, 100) == 0
+    need = lib.awq_search_workspace_bytes(4, 16, 128)
+    assert need > 0
+    assert lib.awq_search_alpha(V(A), V(A), 4, 16, 128, a1, 1, None, V(A), V(A), need, None) == 1
+    assert lib.awq_search_alpha(V(A), V(A), 4, 16, 128, a1, 1, V(A), V(A), V(A), need - 1, None) == 1
+    assert lib.awq_search_alpha(V(A), V(A), 4, 16, 128, anan, 1, V(A), V(A), V(A), need, None) == 1
+    assert lib.awq_search_alpha(V(A), V(A), 4, 16, 128, a1, 0, V(A), V(A), V(A), need, None) == 1
+    assert lib.awq_search_alpha(V(MIS), V(A), 4, 16, 128, a1, 1, V(A), V(A), V(A), need, None) == 3
+    # fused epilogues: I a positive multiple of 16, Nq and Nkv positive, aligned outputs
+    assert lib.awq_w4a16_linear_silu_mul(V(A), V(A), V(A), V(A), V(A), 1, 24, 128, None) == 1
+    assert lib.awq_w4a16_linear_silu_mul(V(A), V(A), V(A), V(A), V(A), 1, 0, 128, None) == 1
+    assert lib.awq_w4a16_linear_qkv(V(A), V(A), V(A), V(A), V(A), V(A), V(A), 1, 64, 0, 128, None) == 1
+    assert lib.awq_w4a16_linear_qkv(V(A), V(A), V(A), V(A), V(A), V(A), None, 1, 64, 8, 128, None) == 1
+    assert lib.awq_w4a16_linear_qkv(V(A), V(A), V(A), V(A), V(A), V(MIS), V(A), 1, 64, 8, 128, None) == 3
     # misaligned pointers
     assert lib.awq_quantize_g128(V(MIS), None, 16, 128, V(A), V(A), V(A), None) == 3
     assert lib.awq_w4a16_gemv(V(A), V(A), V(A), V(A), V(MIS), 1, 16, 128, None) == 3

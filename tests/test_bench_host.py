@@ -40,3 +40,29 @@ def test_every_workload_has_a_bench_config():
             cfg = bench.bench_config(wl, M)
             assert cfg["workload"] == name and cfg["M"] == M
             assert ("decode GEMV" in cfg["step"]) == (M <= 32)
+
+
+def test_exact_step_plan_times_exactly_k_steps():
+    for steps in [1, 3, 20, 49, 50, 51, 100, 2000, 2017]:
+        R, full, rem = bench.exact_step_plan(steps, 50)
+        assert R * full + rem == steps and 0 <= rem < R and R <= 50
+
+
+def test_rotation_covers_four_times_l2():
+    l2 = 126 * 1024 * 1024
+    for set_bytes in [8.7e6, 105e6, 122e6, 600e6]:
+        n = bench.rotation_sets(int(set_bytes), l2)
+        assert n >= 2 and n * set_bytes >= 4 * l2
+
+
+def test_packed_bytes_matches_the_layout():
+    from oracle import awq_oracle as O
+    for N, K in [(4096, 4096), (12288, 4096), (4096, 11008), (300, 384), (28672, 8192)]:
+        words, halves, zb = O.packed_sizes(N, K)
+        assert bench.packed_bytes(N, K) == 4 * words + 2 * halves + zb
+
+
+def test_parse_defaults_and_reference_metric():
+    a = bench.parse_args([])
+    assert a.steps > 0 and a.warmup >= 3 and a.impl == "ours" and a.workload == "llama2_7b_decode_m1"
+    assert "GEMV" in bench.metric_name(1)

@@ -113,6 +113,37 @@ def test_quantize_hand_groups_and_extremes():
     _quant_check(W, s, W.shape[0], 256)
 
 
+def _exhaustive_groups(lo, hi):
+    """Rows of 128-weight groups: each group holds lo and hi (which fix S and z) and 126 fp16 values
+    from [lo, hi]; together the groups hold every finite fp16 value in that interval."""
+    allv = np.arange(0, 65536, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    allv = allv[np.isfinite(allv)]
+    vals = allv[(allv >= np.float16(lo)) & (allv <= np.float16(hi))]
+    vals = np.unique(vals.astype(np.float32)).astype(np.float16)          # -0 and +0 once
+    n = -(-len(vals) // 126)
+    body = np.resize(vals, n * 126).reshape(n, 126)                        # wraps around to fill
+    g = np.empty((n, 128), np.float16)
+    g[:, 0], g[:, 1], g[:, 2:] = np.float16(lo), np.float16(hi), body
+    return g
+
+
+@pytest.mark.parametrize("fold", [False, True])
+def test_quantize_every_fp16_value_over_scale_ranges(fold):
+    """Every finite fp16 value is coded in groups whose bounds fix S across the whole range of
+    scales: the 1e-5 floor (0x000b), subnormal S, S around 1, large S and the full fp16 range.
+    This drives the exact three-operation division and both clamp paths with every operand."""
+    bounds = [(0.0, 0.0), (-1e-6, 1e-6), (-2.0 ** -14, 2.0 ** -13), (-1.0, 1.0), (-7.0, 8.0), (0.5, 3.0),
+              (-9.0, -2.0), (-1000.0, 250.0), (-65504.0, 65504.0)]
+    groups = np.concatenate([_exhaustive_groups(lo, hi) for lo, hi in bounds])
+    # rows of K = 2048 (16 groups); pad the last row with copies of the first group
+    per_row = 16
+    nrows = -(-len(groups) // per_row)
+    groups = np.concatenate([groups, np.repeat(groups[:1], nrows * per_row - len(groups), axis=0)])
+    W = groups.reshape(nrows, per_row * 128)
+    s = np.ones(W.shape[1], np.float32) if fold else None
+    _quant_check(W, s, W.shape[0], W.shape[1])
+
+
 def _full_layer_quant_check(W, s, rows_per_chunk=2048):
     """Quantize a whole layer on the GPU; compare every packed byte with the oracle's codes packed by
     the oracle's packer, chunk by chunk of rows (a tile's codes, scales and zeros are contiguous)."""
@@ -241,21 +272,37 @@ def test_decode_m1_full_size_sampled(layer_idx):
     _full_size_case("llama2_7b_decode_m1", layer_idx, 1, "awq_w4a16_gemv")
 
 
-@pytest.mark.parametrize("layer_idx,M", [(0, 4), (2, 32), (3, 16)])
+@pytest.mark.parametrize("M", [4, 8, 16, 32])
+@pytest.mark.parametrize("layer_idx", [0, 1, 2, 3])
 def test_batched_decode_full_size_sampled(layer_idx, M):
-    _full_size_case("llama2_7b_decode_batched", layer_idx, M, "awq_w4a16_gemv")
+    """Every (layer, M) pair of the Llama-2-7B batched decode set, through the dispatching call."""
+    _full_size_case("llama2_7b_decode_batched", layer_idx, M, "awq_w4a16_linear")
 
 
-@pytest.mark.parametrize("layer_idx,M", [(0, 512), (2, 2048), (3, 4096), (1, 4096)])
+@pytest.mark.parametrize("M", [512, 2048, 4096])
+@pytest.mark.parametrize("layer_idx", [0, 1, 2, 3])
 def test_prefill_full_size_sampled(layer_idx, M):
+    """Every (layer, M) pair of the Llama-3-8B prefill set."""
     _full_size_case("llama3_8b_prefill", layer_idx, M, "awq_w4a16_gemm")
 
 
-@pytest.mark.parametrize("layer_idx,M,fn", [(0, 1, "awq_w4a16_gemv"), (1, 16, "awq_w4a16_gemv"),
-                                            (1, 512, "awq_w4a16_gemm")])
-def test_70b_full_size_sampled(layer_idx, M, fn):
-    _full_size_case("llama2_70b_layers", layer_idx, M, fn)
+@pytest.mark.parametrize("M", [1, 16, 512])
+@pytest.mark.parametrize("layer_idx", [0, 1])
+def test_70b_full_size_sampled(layer_idx, M):
+    """Every (layer, M) pair of the Llama-2-70B set, through the dispatching call."""
+    _full_size_case("llama2_70b_layers", layer_idx, M, "awq_w4a16_linear")
 
+
+@pytest.mark.parametrize("M", [1, 2, 9, 64])
+@pytest.mark.parametrize("N", [16, 200])
+def test_single_group_k128(M, N):
+    """K = 128: one group per row (G = 1, so one padding group per tile), both kernels."""
+    x, W = workloads.random_case(61 + M, M, N, 128)
+    r = O.reference_forward(x, W)
+    for fn in (["awq_w4a16_gemv"] if M <= 32 else []) + ["awq_w4a16_gemm"]:
+        y = _pipeline(x, W, fn)
+        assert_tolerance(y, r["y"], f"{fn} K=128 M={M} N={N}")
+        assert_tight(y, r["y"], what=f"{fn} K=128")
 
 
 # ----------------------------------------------------------------------------- launch chaining

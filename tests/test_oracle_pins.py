@@ -451,3 +451,33 @@ def test_alpha_grid_is_even_over_unit_interval():
     g = O.alpha_grid(20)
     assert g.dtype == np.float32 and g[0] == 0.0 and g[10] == 0.5 and len(g) == 20 and g[-1] < 1.0
     assert np.allclose(np.diff(g.astype(np.float64)), 0.05)
+
+
+# ----------------------------------------------------------------------------
+# fused epilogues
+# ----------------------------------------------------------------------------
+def test_silu_closed_forms():
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    # SiLU(v) -> v for large v, -> 0 for very negative v; SiLU(ln 3) = ln(3) * 3/4
+    assert abs(O.silu(np.array([40.0]))[0] - 40.0) < 1e-12
+    assert abs(O.silu(np.array([-40.0]))[0]) < 1e-15
+    assert abs(O.silu(np.array([np.log(3.0)]))[0] - 0.75 * np.log(3.0)) < 1e-15
+    # odd part: SiLU(v) - SiLU(-v) = v
+    v = np.linspace(-5, 5, 11)
+    assert np.allclose(O.silu(v) - O.silu(-v), v, rtol=0, atol=1e-14)
+
+
+def test_gate_up_silu_pairs_row_i_with_row_i_plus_I():
+    y = np.zeros((2, 6))
+    y[:, :3] = [[0.0, np.log(3.0), 1.0], [2.0, -1.0, 0.5]]
+    y[:, 3:] = [[5.0, 4.0, 0.0], [1.0, 2.0, -2.0]]
+    h = O.gate_up_silu(y)
+    assert h.shape == (2, 3)
+    assert h[0, 0] == 0.0 and abs(h[0, 1] - 3.0 * np.log(3.0)) < 1e-14 and h[0, 2] == 0.0
+    assert abs(h[1, 0] - 2.0 / (1.0 + np.exp(-2.0))) < 1e-15
+
+
+def test_split_qkv_blocks():
+    y = np.arange(2 * 12).reshape(2, 12)
+    q, k, v = O.split_qkv(y, 8, 2)
+    assert q.tolist() == y[:, :8].tolist() and k.tolist() == y[:, 8:10].tolist() and v.tolist() == y[:, 10:].tolist()

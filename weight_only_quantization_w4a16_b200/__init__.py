@@ -14,6 +14,9 @@ Functions (same names as the C ABI):
 * ``awq_w4a16_gemv(x, qweight, scales, zeros, N)`` -> y[M,N] fp16 (M <= 32)
 * ``awq_w4a16_gemm(x, qweight, scales, zeros, N)`` -> y[M,N] fp16
 * ``awq_w4a16_linear(...)``: gemv for M <= 32, gemm otherwise
+* ``awq_w4a16_linear_qkv(x, qweight, scales, zeros, Nq, Nkv)`` -> (q, k, v): fused q/k/v split
+* ``awq_w4a16_linear_silu_mul(x, qweight, scales, zeros, I)`` -> h = SiLU(gate) * up
+* ``awq_search_alpha(x, W, alphas)`` -> (err[n] float64, best index): the AWQ scale search
 * ``awq_poll_device_status()``, test hooks ``awq_debug_set_wait_budget_ns(ns)``,
   ``awq_debug_drop_first_copy(enable)``
 """
@@ -63,6 +66,10 @@ _SIGS = {
     "awq_w4a16_gemm": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_w4a16_linear": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_poll_device_status": ([_VP], _I),
+    "awq_search_workspace_bytes": ([_I, _I, _I], ctypes.c_size_t),
+    "awq_w4a16_linear_qkv": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP], _I),
+    "awq_w4a16_linear_silu_mul": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
+    "awq_search_alpha": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP], _I),
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
     "awq_debug_drop_first_copy": ([_I], _I),
 }
@@ -282,6 +289,77 @@ def awq_w4a16_gemm(x, qweight, scales, zeros, N: int, y=None):
 def awq_w4a16_linear(x, qweight, scales, zeros, N: int, y=None):
     """The decode kernel for small M, the prefill kernel otherwise (the library picks)."""
     return _linear("awq_w4a16_linear", x, qweight, scales, zeros, N, y)
+
+
+def awq_w4a16_linear_qkv(x, qweight, scales, zeros, Nq: int, Nkv: int, out=None):
+    """Fused q/k/v layer (weight rows: Nq query, Nkv key, Nkv value); returns (q, k, v)."""
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    M, K = x.shape
+    N = Nq + 2 * Nkv
+    if out is None:
+        out = tuple(torch.empty((M, n), dtype=torch.float16, device=x.device) for n in (Nq, Nkv, Nkv))
+    _check_packed(qweight, scales, zeros, N, K)
+    for t, n, name in zip(out, (Nq, Nkv, Nkv), ("q", "k", "v")):
+        _need(t, torch.float16, name, 2)
+        if tuple(t.shape) != (M, n):
+            raise ValueError(f"{name} must have shape {(M, n)}")
+    st = load_library().awq_w4a16_linear_qkv(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), *[_ptr(t) for t in out],
+                                             M, Nq, Nkv, K, _stream_ptr())
+    _check("awq_w4a16_linear_qkv", st)
+    return out
+
+
+def awq_w4a16_linear_silu_mul(x, qweight, scales, zeros, I: int, h=None):
+    """Fused gate+up layer (weight rows: I gate, then I up; I % 16 == 0): h = SiLU(gate) * up."""
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    M, K = x.shape
+    if I < 16 or I % 16:
+        raise ValueError("I must be a positive multiple of 16")
+    if h is None:
+        h = torch.empty((M, I), dtype=torch.float16, device=x.device)
+    _check_packed(qweight, scales, zeros, 2 * I, K)
+    _need(h, torch.float16, "h", 2)
+    if tuple(h.shape) != (M, I):
+        raise ValueError(f"h must have shape {(M, I)}")
+    st = load_library().awq_w4a16_linear_silu_mul(_ptr(x), _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(h), M, I,
+                                                  K, _stream_ptr())
+    _check("awq_w4a16_linear_silu_mul", st)
+    return h
+
+
+def awq_search_alpha(x, W, alphas=None, workspace=None):
+    """AWQ scale search: the squared output error of the whole path for every candidate exponent.
+
+    ``alphas`` defaults to an even grid of 20 points over [0, 1). Returns (err, best, alphas) with
+    err a float64 CUDA tensor and best a one-element int32 CUDA tensor (no host synchronization).
+    """
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    _need(W, torch.float16, "W", 2)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError(f"W must have K={K} columns")
+    if alphas is None:
+        alphas = [i / 20.0 for i in range(20)]
+    a = (ctypes.c_float * len(alphas))(*[float(v) for v in alphas])
+    lib = load_library()
+    need = int(lib.awq_search_workspace_bytes(M, N, K))
+    if need == 0:
+        raise ValueError("shape out of range for the search")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _need(workspace, torch.uint8, "workspace", 1)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace must hold {need} bytes")
+    err = torch.empty(len(alphas), dtype=torch.float64, device=x.device)
+    best = torch.empty(1, dtype=torch.int32, device=x.device)
+    st = lib.awq_search_alpha(_ptr(x), _ptr(W), M, N, K, ctypes.cast(a, _VP), len(alphas), _ptr(err), _ptr(best),
+                              _ptr(workspace), workspace.numel(), _stream_ptr())
+    _check("awq_search_alpha", st)
+    return err, best, list(alphas)
 
 
 def awq_poll_device_status() -> int:

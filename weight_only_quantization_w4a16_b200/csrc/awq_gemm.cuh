@@ -32,6 +32,43 @@
 
 namespace awq {
 
+// Epilogue of the linear kernels ("transformers - AWQ" section 3, fused modules):
+//   kEpiPlain  y[M, N]
+//   kEpiSplit3 the fused q/k/v output split into y0 [M, n0], y1 [M, n1], y2 [M, N - n0 - n1]
+//   kEpiSiluMul the fused gate+up layer (weight rows: I gate rows, then I up rows, I % 16 == 0):
+//              h[M, I] = SiLU(gate) * up, written to y0; the prefill kernel loads each 128-row
+//              block as 4 gate tiles and the 4 matching up tiles, interleaved by 16 rows, so a
+//              gate row and its up row sit 16 accumulator lanes apart in one warp
+constexpr int kEpiPlain = 0;
+constexpr int kEpiSplit3 = 1;
+constexpr int kEpiSiluMul = 2;
+struct EpiArgs {
+  __half* y0;
+  __half* y1;
+  __half* y2;
+  int n0, n1;   // kEpiSplit3: widths of y0 and y1 (y2 takes the rest of N)
+};
+
+// Stores one fp32 output of row n (of N), token m, per the epilogue (kEpiPlain / kEpiSplit3).
+template <int EPI>
+__device__ __forceinline__ void epi_store(const EpiArgs& e, int m, long long n, int N, float v) {
+  if (EPI == kEpiSplit3) {
+    if (n < e.n0) {
+      e.y0[static_cast<size_t>(m) * e.n0 + n] = __float2half_rn(v);
+    } else if (n < e.n0 + e.n1) {
+      e.y1[static_cast<size_t>(m) * e.n1 + (n - e.n0)] = __float2half_rn(v);
+    } else {
+      const int n2 = N - e.n0 - e.n1;
+      e.y2[static_cast<size_t>(m) * n2 + (n - e.n0 - e.n1)] = __float2half_rn(v);
+    }
+  } else {
+    e.y0[static_cast<size_t>(m) * N + n] = __float2half_rn(v);
+  }
+}
+
+// SiLU(g) * u in fp32 (SiLU(g) = g / (1 + e^-g)).
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 // CPS: resident CTAs per SM. With 2, each CTA keeps one TMEM accumulator (the other CTA's
 // epilogue and mainloop interleave with its own); with 1, two accumulators let the epilogue of
 // one tile overlap the mainloop of the next.
@@ -44,8 +81,9 @@ struct GemmCfg {
   static constexpr int kB = BT * kKTile * 2;                // x' tile
   static constexpr int kRawQ = kSuperChunkWords * 4;        // 4096 B
   static constexpr int kRawS = 8 * 16 * 2;                  // 256 B
-  static constexpr int kRawZ = 8 * 16;                      // 128 B: zeros of the group pair, 8 tiles
-  static constexpr int kTx = kB + kRawQ + kRawS + kRawZ;
+  static constexpr int kZeroBytes = 8 * 16;                 // 128 B: zeros of the group pair, 8 tiles
+  static constexpr int kRawZ = 256;                         // zeros slot: two 128-byte-aligned halves
+  static constexpr int kTx = kB + kRawQ + kRawS + kZeroBytes;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kA;
   static constexpr int kOffQ = kOffB + STAGES * kB;
@@ -70,11 +108,11 @@ struct GemmCfg {
   static_assert(CPS == 1 || (kSmem + 1024) * 2 <= 233472, "two CTAs per SM must fit in shared memory");
 };
 
-template <int BT, int STAGES, int NDQ, int CPS>
+template <int BT, int STAGES, int NDQ, int CPS, int EPI>
 __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     awq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
-                    __half* __restrict__ y, int M, int N, int K) {
+                    const EpiArgs epi, int M, int N, int K) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,7 +127,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NST = padded_rows(N) / kSuperRows;
+  // kEpiSiluMul: N = 2I rows, P = I/16 tile pairs; super-tile st = gate tiles 4st..4st+3 and up
+  // tiles P + 4st..P + 4st + 3
+  const int P = N / 32;
+  const int NST = EPI == kEpiSiluMul ? ceil_div(P, 4) : padded_rows(N) / kSuperRows;
   const int MTT = (M + BT - 1) / BT;
   const int ntiles = NST * MTT;
   const int KB = K / kKTile;
@@ -137,9 +178,20 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::kTx);
-          tma_load_3d(smem + C::kOffQ + stage * C::kRawQ, &tmap_q, 0, kb, 8 * st, &full[stage]);
-          tma_load_3d(smem + C::kOffS + stage * C::kRawS, &tmap_s, 0, kb >> 1, 8 * st, &full[stage]);
-          tma_load_3d(smem + C::kOffZ + stage * C::kRawZ, &tmap_z, 0, kb >> 2, 8 * st, &full[stage]);
+          if (EPI == kEpiSiluMul) {   // 4-tile boxes: gate tiles to slots 0..3, up tiles to slots 4..7
+            tma_load_3d(smem + C::kOffQ + stage * C::kRawQ, &tmap_q, 0, kb, 4 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffQ + stage * C::kRawQ + C::kRawQ / 2, &tmap_q, 0, kb, P + 4 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffS + stage * C::kRawS, &tmap_s, 0, kb >> 1, 4 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffS + stage * C::kRawS + C::kRawS / 2, &tmap_s, 0, kb >> 1, P + 4 * st,
+                        &full[stage]);
+            tma_load_3d(smem + C::kOffZ + stage * C::kRawZ, &tmap_z, 0, kb >> 2, 4 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffZ + stage * C::kRawZ + 128, &tmap_z, 0, kb >> 2, P + 4 * st,
+                        &full[stage]);
+          } else {
+            tma_load_3d(smem + C::kOffQ + stage * C::kRawQ, &tmap_q, 0, kb, 8 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffS + stage * C::kRawS, &tmap_s, 0, kb >> 1, 8 * st, &full[stage]);
+            tma_load_3d(smem + C::kOffZ + stage * C::kRawZ, &tmap_z, 0, kb >> 2, 8 * st, &full[stage]);
+          }
           tma_load_2d(smem + C::kOffB + stage * C::kB, &tmap_x, kb * kKTile, mt * BT, &full[stage]);
           issued_mask |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -196,7 +248,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget)) { ok = false; break; }
+        // warp-uniform result: the code below needs the whole warp
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, s_abort, budget))) { ok = false; break; }
         const uint32_t* rq = reinterpret_cast<const uint32_t*>(smem + C::kOffQ + stage * C::kRawQ);
         const uint32_t* rs = reinterpret_cast<const uint32_t*>(smem + C::kOffS + stage * C::kRawS);
         const uint8_t* rz = smem + C::kOffZ + stage * C::kRawZ;
@@ -205,9 +258,13 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
         for (int u = 0; u < 8 / NDQ; ++u) {
           const int c = warp * 32 + lane + u * 32 * NDQ;   // (16-row tile, lane) chunk
           const int nt = c >> 5, lw = c & 31, r = lw >> 2, t = lw & 3;
-          const uint4 words = *reinterpret_cast<const uint4*>(rq + nt * kChunkWords + lw * 4);
-          const uint32_t sp = rs[nt * 8 + r];                        // (S_r, S_{r+8})
-          const uint32_t zb = rz[nt * 16 + ((kb >> 1) & 1) * 8 + r];
+          // 16-row block nt of the A tile comes from shared-memory slot sl (kEpiSiluMul interleaves
+          // gate and up tiles: blocks 2e and 2e+1 are gate tile e and up tile e)
+          const int sl = EPI == kEpiSiluMul ? ((nt & 1) ? 4 + (nt >> 1) : (nt >> 1)) : nt;
+          const uint4 words = *reinterpret_cast<const uint4*>(rq + sl * kChunkWords + lw * 4);
+          const uint32_t sp = rs[sl * 8 + r];                        // (S_r, S_{r+8})
+          const int zoff = (EPI == kEpiSiluMul && sl >= 4) ? 128 + (sl - 4) * 16 : sl * 16;
+          const uint32_t zb = rz[zoff + ((kb >> 1) & 1) * 8 + r];
           const uint32_t s_r = __byte_perm(sp, 0, 0x1010);          // (S_r, S_r)
           const uint32_t s_r8 = __byte_perm(sp, 0, 0x3232);         // (S_{r+8}, S_{r+8})
           const uint32_t za = 0x64006400u | ((zb & 0xFu) * 0x00010001u);
@@ -242,21 +299,32 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
       const int st = tile % NST, mt = tile / NST;
       const int b = it % C::kNAcc;
       const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
-      if (!mbar_wait_bounded(&accfull[b], use & 1, s_abort, budget)) { ok = false; break; }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&accfull[b], use & 1, s_abort, budget))) { ok = false; break; }
       tc_fence_after();
       const int n = st * kSuperRows + 32 * e + lane;
       const bool n_ok = n < N;
+      // kEpiSiluMul: lanes 0..15 of this quarter hold gate row i, lanes 16..31 the up row i
+      const int i_gu = 16 * (4 * st + e) + (lane & 15);
 #pragma unroll 1
       for (int cc = 0; cc < BT / 32; ++cc) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * e) << 16) + static_cast<uint32_t>(b * BT + 32 * cc), v);
         tc_wait_ld();
         const int mb = mt * BT + 32 * cc;
-        if (n_ok) {
+        if (EPI == kEpiSiluMul) {
+          const int I = N / 2;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float g = __uint_as_float(v[j]);
+            const float u = __shfl_down_sync(0xFFFFFFFFu, g, 16);
+            const int m = mb + j;
+            if (lane < 16 && i_gu < I && m < M) epi.y0[static_cast<size_t>(m) * I + i_gu] = __float2half_rn(silu_mul(g, u));
+          }
+        } else if (n_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int m = mb + j;
-            if (m < M) y[static_cast<size_t>(m) * N + n] = __float2half_rn(__uint_as_float(v[j]));
+            if (m < M) epi_store<EPI>(epi, m, n, N, __uint_as_float(v[j]));
           }
         }
       }

@@ -33,6 +33,7 @@
 #include <cooperative_groups.h>
 
 #include "awq_common.cuh"
+#include "awq_gemm.cuh"
 
 namespace awq {
 
@@ -61,6 +62,11 @@ struct GemvArgs {
   int off_scales, off_zeros, off_x;   // offsets inside a stage
   int x_box_bytes;          // bytes of the stage's x' box (4*SB k-tiles x M tokens x 128)
   int x_swizzle;            // the x' box uses the 128-byte swizzle (M > 2)
+  // fused epilogues (ring form): kEpiSplit3 writes y, y1, y2 with widths n0, n1, N - n0 - n1;
+  // kEpiSiluMul pairs logical unit 2j (gate tile j) with 2j + 1 (up tile P + j), P = N / 32
+  __half* y1;
+  __half* y2;
+  int n0, n1;
 };
 
 // Worker (warp) w of W that holds item i of a cluster's L items, when worker w owns items
@@ -440,16 +446,273 @@ __global__ void __launch_bounds__(GemvCfg<MT, NT, CW, D, SB>::kThreads, 1)
           off = (static_cast<int>(w % CW) * R + (ur - static_cast<int>(aw / G2))) * rec_elems;
         }
       }
-      for (int e = lane; e < per_unit; e += 32) {
-        const int m = e / (NT * 16), row = e - m * (NT * 16);
+      // every lane runs every iteration (the shuffles need the whole warp); lanes past the unit's
+      // outputs only skip the loads and the store
+      for (int e0 = 0; e0 < per_unit; e0 += 32) {
+        const int e = e0 + lane;
+        const bool live = e < per_unit;
+        const int m = live ? e / (NT * 16) : 0, row = live ? e - m * (NT * 16) : 0;
         float v = 0.f;
         for (int c = 0; c < ncontrib; ++c) {
           const int cc = __shfl_sync(0xFFFFFFFFu, cta, c);
           const int oo = __shfl_sync(0xFFFFFFFFu, off, c);
-          if (cc >= 0) v += cluster.map_shared_rank(rec_all, cc)[oo + row * M + m];
+          if (live && cc >= 0) v += cluster.map_shared_rank(rec_all, cc)[oo + row * M + m];
         }
         const size_t n = ybase + row;
-        if (n < static_cast<size_t>(a.N)) a.y[static_cast<size_t>(m) * a.N + n] = __float2half_rn(v);
+        if (live && n < static_cast<size_t>(a.N)) a.y[static_cast<size_t>(m) * a.N + n] = __float2half_rn(v);
+      }
+    }
+  }
+  // no CTA leaves while another may still read its shared memory
+  cluster_arrive();
+  cluster_wait();
+}
+
+
+// ------------------------------------------------------------------------------------
+// Shared-ring form: one producer lane streams the CTA's contiguous item range (with 16-row
+// units a CTA's range is one contiguous byte range of each packed array in layout v2) into a
+// ring of S stages of up to SB group pairs of one tile; CW consumer warps split each stage's
+// group pairs. Every consumer warp writes a record for every unit of the CTA's range (zeros
+// where it had no item), the CTA adds its warps' records in warp order, and the cluster adds
+// the CTAs' records of each unit in rank order through distributed shared memory.
+template <int CW, int SB>
+struct GemvRingCfg {
+  static constexpr int kThreads = 32 * (CW + 1);
+  static constexpr int kCodes = SB * 2048;
+  static constexpr int kScales = SB * 64;
+  static constexpr int kZeros = SB * 16;
+};
+
+template <int MT, int CW, int S, int SB, int NACC, bool kSumX, int EPI>
+__global__ void __launch_bounds__(GemvRingCfg<CW, SB>::kThreads, 1)
+    awq_gemv_ring_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemvArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int cid = static_cast<int>(blockIdx.x) / CL;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = a.M, G2 = a.g2;
+  const int rec_elems = 16 * M;   // floats per record (one 16-row unit)
+  const int R = a.rec_per_warp;   // units a CTA's range touches at most
+  float* rec_all = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * a.stage_bytes);   // [CW][R][16][M]
+  uint64_t* full = reinterpret_cast<uint64_t*>(rec_all + static_cast<size_t>(CW) * R * rec_elems);
+  uint64_t* empty = full + S;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + S);
+
+  // ---- this cluster's units and this CTA's item range (kEpiSiluMul: whole gate/up unit pairs)
+  const int P = a.N / 32;
+  const long long upc = EPI == kEpiSiluMul ? 2 : 1;
+  const long long u0 = upc * (static_cast<long long>(cid) * (a.units / upc) / a.clusters);
+  const long long u1 = upc * (static_cast<long long>(cid + 1) * (a.units / upc) / a.clusters);
+  const long long L = (u1 - u0) * G2;
+  const long long i0 = static_cast<long long>(rank) * L / CL, i1 = static_cast<long long>(rank + 1) * L / CL;
+  // physical tile of a (logical) unit
+  auto tile_of = [&](int u) -> int { return EPI == kEpiSiluMul ? ((u & 1) ? P + (u >> 1) : (u >> 1)) : u; };
+
+  if (threadIdx.x == 0) {
+    for (int d = 0; d < S; ++d) {
+      mbar_init(&full[d], 1);
+      mbar_init(&empty[d], CW);
+    }
+    *s_abort = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  const unsigned long long budget = g_wait_budget_ns;
+
+  struct Cursor {
+    long long it;   // item index within the cluster's range
+    int u;          // unit (absolute)
+    int p;          // group pair within the unit
+  };
+  auto stage_np = [&](const Cursor& c) -> int {
+    const long long left = i1 - c.it;
+    return static_cast<int>(min(static_cast<long long>(min(SB, G2 - c.p)), left));
+  };
+  auto advance = [&](Cursor& c, int np) {
+    c.it += np;
+    c.p += np;
+    if (c.p == G2) { c.p = 0; ++c.u; }
+  };
+  const Cursor start = {i0, static_cast<int>(u0 + i0 / G2), static_cast<int>(i0 % G2)};
+  const bool drop0 = g_debug_drop_first_copy != 0;
+  bool ok = true;
+
+  if (warp == CW) {
+    // ---------------------------------------------------------------- producer lane
+    if (lane == 0) {
+      auto issue_weights = [&](int slot, const Cursor& c) {
+        const int np = stage_np(c);
+        uint8_t* sb = smem + static_cast<size_t>(slot) * a.stage_bytes;
+        mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(np * (2048 + 64 + 16) + a.x_box_bytes));
+        const size_t tp = static_cast<size_t>(tile_of(c.u)) * G2 + c.p;   // (tile, pair) index
+        bulk_g2s(sb, a.qweight + tp * 2048, np * 2048, &full[slot]);
+        bulk_g2s(sb + a.off_scales, a.scales + tp * 64, np * 64, &full[slot]);
+        bulk_g2s(sb + a.off_zeros, a.zeros + tp * 16, np * 16, &full[slot]);
+      };
+      auto issue_x = [&](int slot, const Cursor& c) {
+        tma_load_3d(smem + static_cast<size_t>(slot) * a.stage_bytes + a.off_x, &tmap_x, 0, 0, 4 * c.p, &full[slot]);
+      };
+      // first ring pass of weights before waiting on the previous kernel
+      Cursor isc = start;
+      int npro = 0;
+      for (; npro < S && isc.it < i1; ++npro) {
+        if (!(drop0 && npro == 0)) issue_weights(npro, isc);
+        advance(isc, stage_np(isc));
+      }
+      if (i0 < i1) tma_prefetch_desc(&tmap_x);
+      pdl_wait();
+      {
+        Cursor c = start;
+        for (int s = 0; s < npro; ++s) {
+          if (!(drop0 && s == 0)) issue_x(s, c);
+          advance(c, stage_np(c));
+        }
+      }
+      int slot = 0;
+      uint32_t phase = 0;
+      for (int s = npro; isc.it < i1; ++s) {
+        // refill the slot of stage s - S once its consumers have released it
+        if (!mbar_wait_bounded(&empty[slot], phase, s_abort, budget)) { ok = false; break; }
+        issue_weights(slot, isc);
+        issue_x(slot, isc);
+        advance(isc, stage_np(isc));
+        if (++slot == S) { slot = 0; phase ^= 1; }
+      }
+      // drain: the last S stages this lane issued may still be in flight if the consumers stopped
+      // early; wait for each (their phases are the most recent of their slots)
+      int n_issued = 0;
+      for (Cursor q = start; q.it < isc.it; advance(q, stage_np(q))) ++n_issued;
+      int never = 0;
+      for (int s2 = max(0, n_issued - S); s2 < n_issued; ++s2)
+        if (!(drop0 && s2 == 0)) mbar_wait_bounded(&full[s2 % S], static_cast<uint32_t>((s2 / S) & 1), &never,
+                                                   kDrainBudgetNs);
+    }
+  } else {
+    // ---------------------------------------------------------------- consumer warps
+    pdl_wait();
+    const int r = lane >> 2, t = lane & 3;
+    const bool swz = a.x_swizzle != 0;
+    float acc[1][MT][4];
+#pragma unroll
+    for (int j = 0; j < MT; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[0][j][c] = 0.f;
+    float* rec = rec_all + static_cast<size_t>(warp) * R * rec_elems;
+    int ri = 0;
+    auto flush = [&]() {
+      float* pr = rec + static_cast<size_t>(ri) * rec_elems;
+#pragma unroll
+      for (int j = 0; j < MT; ++j)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int m = 8 * j + 2 * t + (c & 1);
+          const int row = r + 8 * (c >> 1);
+          if (m < M) pr[row * M + m] = acc[0][j][c];
+          acc[0][j][c] = 0.f;
+        }
+    };
+    int slot = 0;
+    uint32_t phase = 0;
+    Cursor cs = start;
+    while (cs.it < i1) {
+      const int np = stage_np(cs);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[slot], phase, s_abort, budget));
+      if (!ok) break;
+      const uint8_t* sb = smem + static_cast<size_t>(slot) * a.stage_bytes;
+#pragma unroll
+      for (int pi = 0; pi < (SB + CW - 1) / CW; ++pi) {
+        const int pp = warp + pi * CW;
+        if (pp < np) {
+#pragma unroll
+          for (int gg = 0; gg < 2; ++gg) {
+            uint4 xv[2][MT][2];
+            uint4 cw[2][1];
+            uint32_t sv[1], zz[1];
+            float sx[2] = {0.f, 0.f};
+            if (kSumX) gemv_group_xsums(sx, sb + a.off_x, 4 * pp + 2 * gg, M, lane);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              gemv_load_x<MT>(xv[kk], sb + a.off_x, 4 * pp + 2 * gg + kk, M, r, t, swz);
+              cw[kk][0] = *reinterpret_cast<const uint4*>(sb + pp * 2048 + (2 * gg + kk) * 512 + lane * 16);
+            }
+            sv[0] = *reinterpret_cast<const uint32_t*>(sb + a.off_scales + pp * 64 + gg * 32 + r * 4);
+            zz[0] = sb[a.off_zeros + pp * 16 + gg * 8 + r];
+            gemv_group<MT, 1, NACC, kSumX>(acc, cw, xv, sv, zz, sx);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      const int u_before = cs.u;
+      advance(cs, np);
+      if (cs.u != u_before && cs.it < i1) {   // the next stage starts a new unit: record this one
+        flush();
+        ++ri;
+      }
+      if (++slot == S) { slot = 0; phase ^= 1; }
+    }
+    if (ok && i0 < i1) flush();
+  }
+
+  // ---- the CTA adds its consumer warps' records, in warp order (all threads of the CTA)
+  __syncthreads();
+  if (*s_abort == 0) {
+    const int n_rec = (i0 < i1) ? static_cast<int>((i1 - 1) / G2 - i0 / G2) + 1 : 0;
+    for (int e = threadIdx.x; e < n_rec * rec_elems; e += blockDim.x) {
+      float v = 0.f;
+      for (int w = 0; w < CW; ++w) v += rec_all[static_cast<size_t>(w) * R * rec_elems + e];
+      rec_all[e] = v;   // warp 0's records now hold the CTA's sums
+    }
+  }
+  // ---- cluster reduction: each output is the sum of the records of the CTAs that touched its
+  // unit, in rank order. One warp per unit (per gate/up pair with kEpiSiluMul).
+  cluster_arrive();
+  cluster_wait();
+  if (*s_abort == 0) {
+    const uint32_t Lu = static_cast<uint32_t>(L), CLu = static_cast<uint32_t>(CL);
+    const int nunits = static_cast<int>(u1 - u0);
+    const int nwarps = CW + 1;
+    // the sum over the contributing CTAs of element (row, m) of relative unit ur
+    auto unit_sum = [&](int ur, int row, int m) -> float {
+      const uint32_t first = static_cast<uint32_t>(ur) * G2, last = first + G2 - 1;
+      const uint32_t cf = ((first + 1) * CLu - 1) / Lu, cl_ = ((last + 1) * CLu - 1) / Lu;
+      float v = 0.f;
+      for (uint32_t c = cf; c <= cl_; ++c) {
+        const uint32_t ac = c * Lu / CLu, bc = (c + 1) * Lu / CLu;
+        if (bc == ac) continue;
+        const int rr = ur - static_cast<int>(ac / G2);
+        v += cluster.map_shared_rank(rec_all, static_cast<int>(c))[rr * rec_elems + row * M + m];
+      }
+      return v;
+    };
+    if (EPI == kEpiSiluMul) {
+      const int I = a.N / 2;
+      for (int pr = rank * nwarps + warp; 2 * pr < nunits; pr += CL * nwarps) {
+        const int j = static_cast<int>(u0 / 2) + pr;   // gate tile j, up tile P + j
+        for (int e = lane; e < rec_elems; e += 32) {
+          const int row = e / M, m = e - row * M;
+          const float g = unit_sum(2 * pr, row, m), u = unit_sum(2 * pr + 1, row, m);
+          const int i = 16 * j + row;
+          if (i < I) a.y[static_cast<size_t>(m) * I + i] = __float2half_rn(silu_mul(g, u));
+        }
+      }
+    } else {
+      EpiArgs epi = {a.y, a.y1, a.y2, a.n0, a.n1};
+      for (int ur = rank * nwarps + warp; ur < nunits; ur += CL * nwarps) {
+        const long long nbase = static_cast<long long>(u0 + ur) * 16;
+        for (int e = lane; e < rec_elems; e += 32) {
+          const int row = e / M, m = e - row * M;
+          const float v = unit_sum(ur, row, m);
+          const long long n = nbase + row;
+          if (n < a.N) epi_store<EPI>(epi, m, n, a.N, v);
+        }
       }
     }
   }

@@ -17,6 +17,7 @@
 #include "awq_gemm.cuh"
 #include "awq_gemv.cuh"
 #include "awq_quant.cuh"
+#include "awq_search.cuh"
 #include "awq_w4a16.h"
 
 namespace awq {
@@ -111,7 +112,8 @@ awq_status_t make_x_map(CUtensorMap* map, const void* x, int M, int K, int BT) {
 //   scales uint16 {16, 2*G2 groups, ntiles}         box {16, 1, 8}
 //   zeros  uint8  {16, G2 pairs, ntiles}            box {16, 1, 8}
 awq_status_t make_weight_maps(CUtensorMap* qm, CUtensorMap* sm, CUtensorMap* zm, const void* qw, const void* sc,
-                              const void* zr, int N, int K) {
+                              const void* zr, int N, int K, int box_tiles = 8) {
+  const cuuint32_t bt = static_cast<cuuint32_t>(box_tiles);
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return AWQ_ERR_CUDA;
   const cuuint64_t nt = static_cast<cuuint64_t>(ceil_div(N, kTileRows));
@@ -120,7 +122,7 @@ awq_status_t make_weight_maps(CUtensorMap* qm, CUtensorMap* sm, CUtensorMap* zm,
   {
     const cuuint64_t dims[3] = {128, 4 * g2, nt};
     const cuuint64_t strides[2] = {512, 4 * g2 * 512};
-    const cuuint32_t box[3] = {128, 1, 8};
+    const cuuint32_t box[3] = {128, 1, bt};
     if (enc(qm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(qw), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -129,7 +131,7 @@ awq_status_t make_weight_maps(CUtensorMap* qm, CUtensorMap* sm, CUtensorMap* zm,
   {
     const cuuint64_t dims[3] = {16, 2 * g2, nt};
     const cuuint64_t strides[2] = {32, 2 * g2 * 32};
-    const cuuint32_t box[3] = {16, 1, 8};
+    const cuuint32_t box[3] = {16, 1, bt};
     if (enc(sm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(sc), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -138,7 +140,7 @@ awq_status_t make_weight_maps(CUtensorMap* qm, CUtensorMap* sm, CUtensorMap* zm,
   {
     const cuuint64_t dims[3] = {16, g2, nt};
     const cuuint64_t strides[2] = {16, g2 * 16};
-    const cuuint32_t box[3] = {16, 1, 8};
+    const cuuint32_t box[3] = {16, 1, bt};
     if (enc(zm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(zr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -322,6 +324,95 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
                    a);
 }
 
+// The shared-ring decode form: CL-CTA clusters over 16-row units, each CTA a contiguous item range
+// streamed by one producer lane into S stages of up to SB group pairs; CW consumer warps.
+template <int MT, int CW, int S, int SB, int NACC = 4, bool kSumX = false, int EPI = kEpiPlain>
+awq_status_t launch_gemv_ring_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                                  const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  using Cfg = GemvRingCfg<CW, SB>;
+  static_assert(!kSumX || MT == 1, "activation sums are taken for tokens 0 and 1 only");
+  auto kernel = awq_gemv_ring_kernel<MT, CW, S, SB, NACC, kSumX, EPI>;
+  constexpr int kMaxSmem = 227 * 1024;
+  static std::atomic<uint64_t> smem_done{0};
+  awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
+  if (st != AWQ_OK) return st;
+  GemvArgs a = {};
+  a.qweight = reinterpret_cast<const uint8_t*>(qw);
+  a.scales = reinterpret_cast<const uint8_t*>(sc);
+  a.zeros = zr;
+  a.y = epi.y0;
+  a.y1 = epi.y1;
+  a.y2 = epi.y2;
+  a.n0 = epi.n0;
+  a.n1 = epi.n1;
+  a.M = M;
+  a.N = N;
+  a.ntiles = ceil_div(N, kTileRows);
+  a.g2 = ceil_div(K / kGroup, 2);
+  a.units = EPI == kEpiSiluMul ? 2 * (N / 32) : a.ntiles;
+  const int upc = EPI == kEpiSiluMul ? 2 : 1;   // units per indivisible cluster share
+  const bool swz = M > 2;
+  a.x_swizzle = swz ? 1 : 0;
+  a.off_scales = Cfg::kCodes;
+  a.off_zeros = a.off_scales + Cfg::kScales;
+  a.off_x = round_up(a.off_zeros + Cfg::kZeros, swz ? 1024 : 128);
+  a.x_box_bytes = 4 * SB * M * 128;
+  a.stage_bytes = round_up(a.off_x + a.x_box_bytes, swz ? 1024 : 128);
+  CUtensorMap map;
+  st = make_x_map_decode(&map, x, M, K, 4 * SB, swz);
+  if (st != AWQ_OK) return st;
+  const int shares = a.units / upc;
+  int cl = AWQ_GEMV_CL;
+  while (cl > 1 && shares < cl) cl /= 2;
+  int clusters = std::max(1, std::min(num_sms / cl, shares));
+  auto records = [&](int C) {
+    int R = 1;
+    for (int c = 0; c < C; ++c) {
+      const long long u0 = upc * (static_cast<long long>(c) * shares / C);
+      const long long u1 = upc * (static_cast<long long>(c + 1) * shares / C);
+      const long long L = (u1 - u0) * a.g2;
+      for (int r = 0; r < cl; ++r) {
+        const long long lo = r * L / cl, hi = (r + 1) * L / cl;
+        if (hi > lo) R = std::max(R, static_cast<int>((hi - 1) / a.g2 - lo / a.g2 + 1));
+      }
+    }
+    return R;
+  };
+  auto smem_of = [&](int R) {
+    return static_cast<size_t>(S) * a.stage_bytes + static_cast<size_t>(CW) * R * kTileRows * M * 4 +
+           static_cast<size_t>(2 * S) * 8 + 16 + 1024;
+  };
+  int R = records(clusters);
+  if (smem_of(R) > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
+  static ClusterOccCache cache;
+  const int fit = max_active_clusters(kernel, Cfg::kThreads, smem_of(R), cl, dev, cache);
+  if (fit < 1) return AWQ_ERR_UNSUPPORTED;
+  if (clusters > fit) {
+    clusters = fit;
+    R = records(clusters);
+    if (smem_of(R) > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
+  }
+  a.clusters = clusters;
+  a.rec_per_warp = R;
+  return launch_ex(kernel, dim3(clusters * cl, 1, 1), dim3(Cfg::kThreads, 1, 1), dim3(cl, 1, 1), smem_of(R), stream,
+                   map, a);
+}
+
+// The ring form with a fused epilogue for any M <= 32 (the stage shrinks as the x' box grows).
+template <int EPI>
+awq_status_t launch_gemv_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  switch ((M + 7) / 8) {
+    case 1:
+      if (M <= 2)
+        return launch_gemv_ring_cfg<1, 8, 4, 8, 4, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+      return launch_gemv_ring_cfg<1, 8, 4, 4, 4, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    case 2: return launch_gemv_ring_cfg<2, 4, 3, 4, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    case 3: return launch_gemv_ring_cfg<3, 4, 3, 2, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    default: return launch_gemv_ring_cfg<4, 4, 3, 2, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+  }
+}
+
 // Compile-time tuning of the decode kernel per token tile: warps per CTA, ring stages per warp,
 // group pairs per stage, accumulator chains, and the M <= 2 form (codes as subnormals, zero
 // point through the activation sums).
@@ -341,14 +432,42 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
 #define AWQ_GEMV_SUMX 0
 #endif
 
+#ifndef AWQ_GEMV_KIND
+#define AWQ_GEMV_KIND 2
+#endif
+#ifndef AWQ_GEMVR_CW
+#define AWQ_GEMVR_CW 8
+#endif
+#ifndef AWQ_GEMVR_S
+#define AWQ_GEMVR_S 4
+#endif
+#ifndef AWQ_GEMVR_SB
+#define AWQ_GEMVR_SB 8
+#endif
+
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
   const int mt = (M + 7) / 8;
+  const EpiArgs epi = {y, nullptr, nullptr, 0, 0};
   switch (mt) {
     case 1:
+      if (AWQ_GEMV_KIND == 2) {
+        if (AWQ_GEMV_SUMX && M <= 2)
+          return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, AWQ_GEMVR_S, AWQ_GEMVR_SB, AWQ_GEMV1_NACC, true>(
+              x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+        if (M <= 2)
+          return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, AWQ_GEMVR_S, AWQ_GEMVR_SB, AWQ_GEMV1_NACC>(
+              x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+        // 3 <= M <= 8: the x' box grows with M, so stages hold fewer group pairs
+        return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, 4, 4, AWQ_GEMV1_NACC>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
+                                                                            stream);
+      }
       if (AWQ_GEMV_SUMX && M <= 2)
         return launch_gemv_cfg<1, 1, AWQ_GEMV1_CW, AWQ_GEMV1_D, AWQ_GEMV1_SB, AWQ_GEMV1_NACC, true>(
             x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      if (M <= 2)
+        return launch_gemv_cfg<1, 1, AWQ_GEMV1_CW, AWQ_GEMV1_D, AWQ_GEMV1_SB, AWQ_GEMV1_NACC>(x, qw, sc, zr, y, M, N,
+                                                                                            K, dev, num_sms, stream);
       // 3 <= M <= 8: the x' box grows with M, so stages hold one group pair
       return launch_gemv_cfg<1, 1, 8, 2, 1, AWQ_GEMV1_NACC>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
     case 2: return launch_gemv_cfg<2, 2, 4, 3, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
@@ -358,23 +477,24 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
-template <int BT, int STAGES, int NDQ, int CPS = 1>
-awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
-                             int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+template <int BT, int STAGES, int NDQ, int CPS = 1, int EPI = kEpiPlain>
+awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS>;
-  auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS>;
+  auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS, EPI>;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, C::kSmem, dev, smem_done);
   if (st != AWQ_OK) return st;
   CUtensorMap xmap, qmap, smap, zmap;
   st = make_x_map(&xmap, x, M, K, BT);
   if (st != AWQ_OK) return st;
-  st = make_weight_maps(&qmap, &smap, &zmap, qw, sc, zr, N, K);
+  st = make_weight_maps(&qmap, &smap, &zmap, qw, sc, zr, N, K, EPI == kEpiSiluMul ? 4 : 8);
   if (st != AWQ_OK) return st;
-  const long long tiles = static_cast<long long>(padded_rows(N) / kSuperRows) * ((M + BT - 1) / BT);
+  const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
+  const long long tiles = nst * ((M + BT - 1) / BT);
   const int grid = static_cast<int>(std::min<long long>(tiles, static_cast<long long>(CPS) * num_sms));
   return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), dim3(0, 0, 0), C::kSmem, stream, xmap, qmap,
-                   smap, zmap, y, M, N, K);
+                   smap, zmap, epi, M, N, K);
 }
 
 // Compile-time tuning of the prefill kernel: dequantization warps, ring stages per token tile
@@ -392,16 +512,17 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 #define AWQ_GEMM_S64 7
 #endif
 
-awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
-                         int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  if (M <= 32) return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+template <int EPI>
+awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  if (M <= 32) return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
   if (M <= 64)
-    return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+    return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
   // Token tile by a round model: the persistent CTAs (one per SM) take tiles round-robin, so a
   // launch costs ceil(tiles / SMs) rounds, and a tile's time grows only slowly with BT because
   // dequantizing its 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted
   // on the Llama-3-8B prefill and Llama-2-70B layers at M = 512 and 2048).
-  const long long nst = padded_rows(N) / kSuperRows;
+  const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
   int best_bt = 64;
   double best = 1e300;
   for (int bt : {256, 128, 64}) {
@@ -414,12 +535,20 @@ awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, 
 #endif
   switch (best_bt) {
     case 256:
-      return launch_gemm_cfg<256, AWQ_GEMM_S256, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      return launch_gemm_cfg<256, AWQ_GEMM_S256, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
+                                                                      stream);
     case 128:
-      return launch_gemm_cfg<128, AWQ_GEMM_S128, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      return launch_gemm_cfg<128, AWQ_GEMM_S128, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
+                                                                      stream);
     default:
-      return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
+      return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
   }
+}
+
+awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
+                         int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  EpiArgs epi = {y, nullptr, nullptr, 0, 0};
+  return launch_gemm_epi<kEpiPlain>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
 }
 
 // Rows are limited so that every count below fits an int: N <= 2^31 - 2^7 and N * K <= 2^34.
@@ -440,6 +569,31 @@ awq_status_t check_linear_args(const void* x, const void* qw, const void* sc, co
 // Packed sizes of layout v2: per (16-row tile, group pair) 2048 + 64 + 16 bytes.
 inline size_t tile_pairs(int N, int K) {
   return static_cast<size_t>(ceil_div(N, kTileRows)) * static_cast<size_t>(ceil_div(K / kGroup, 2));
+}
+
+// Workspace of the scale search, each piece 256-byte aligned: y_ref fp32 [M,N], y fp16 [M,N], s fp32 [K],
+// x' fp16 [M,K], the packed weights, and the error reduction's partial sums.
+struct SearchWs {
+  size_t y_ref, y, s, xs, qw, sc, zr, partial, total;
+};
+inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+SearchWs search_ws(int M, int N, int K) {
+  SearchWs w{};
+  size_t o = 0;
+  w.y_ref = o; o = align256(o + static_cast<size_t>(M) * N * 4);
+  w.y = o; o = align256(o + static_cast<size_t>(M) * N * 2);
+  w.s = o; o = align256(o + static_cast<size_t>(K) * 4);
+  w.xs = o; o = align256(o + static_cast<size_t>(M) * K * 2);
+  w.qw = o; o = align256(o + tile_pairs(N, K) * kPairCodeBytes);
+  w.sc = o; o = align256(o + tile_pairs(N, K) * kPairScaleBytes);
+  w.zr = o; o = align256(o + tile_pairs(N, K) * kPairZeroBytes);
+  w.partial = o; o = align256(o + static_cast<size_t>(kSearchMaxBlocks) * 8);
+  w.total = o;
+  return w;
+}
+inline bool search_shape_ok(int M, int N, int K) {
+  return M >= 1 && M <= 65535 * 16 && K >= kGroup && K % kGroup == 0 && rows_ok(N, K) &&
+         static_cast<long long>(M) * K <= (1ll << 31) - 1 && static_cast<long long>(M) * N <= (1ll << 31) - 1;
 }
 
 }  // namespace
@@ -584,6 +738,93 @@ awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const 
                               uint16_t* y, int M, int N, int K, awq_stream_t stream) {
   if (M >= 1 && M <= 32) return awq_w4a16_gemv(x, qweight, scales, zeros, y, M, N, K, stream);
   return awq_w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream);
+}
+
+size_t awq_search_workspace_bytes(int M, int N, int K) {
+  if (!search_shape_ok(M, N, K)) return 0;
+  return search_ws(M, N, K).total;
+}
+
+awq_status_t awq_search_alpha(const uint16_t* x, const uint16_t* W, int M, int N, int K, const float* alphas,
+                              int n_alpha, double* err, int* best, void* workspace, size_t workspace_bytes,
+                              awq_stream_t stream) {
+  if (!x || !W || !alphas || !err || !best || !workspace) return AWQ_ERR_INVALID_ARG;
+  if (!search_shape_ok(M, N, K) || n_alpha < 1 || n_alpha > 4096) return AWQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_alpha; ++i)
+    if (!(alphas[i] == alphas[i]) || alphas[i] > 3.0e38f || alphas[i] < -3.0e38f) return AWQ_ERR_INVALID_ARG;
+  const SearchWs w = search_ws(M, N, K);
+  if (workspace_bytes < w.total) return AWQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(err) & 7u) ||
+      (reinterpret_cast<uintptr_t>(best) & 3u))
+    return AWQ_ERR_MISALIGNED;
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* y_ref = reinterpret_cast<float*>(ws + w.y_ref);
+  uint16_t* y = reinterpret_cast<uint16_t*>(ws + w.y);
+  float* s = reinterpret_cast<float*>(ws + w.s);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + w.xs);
+  uint32_t* qw = reinterpret_cast<uint32_t*>(ws + w.qw);
+  uint16_t* sc = reinterpret_cast<uint16_t*>(ws + w.sc);
+  uint8_t* zr = ws + w.zr;
+  double* partial = reinterpret_cast<double*>(ws + w.partial);
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  // the layer's unquantized output on the calibration rows, once
+  st = launch_ex(awq_ref_gemm_kernel, dim3(static_cast<unsigned>(ceil_div(N, 128)), static_cast<unsigned>(ceil_div(M, 16)), 1),
+                 dim3(128, 1, 1), dim3(0, 0, 0), 0, cs, reinterpret_cast<const __half*>(x),
+                 reinterpret_cast<const __half*>(W), y_ref, M, N, K);
+  if (st != AWQ_OK) return st;
+  const long long count = static_cast<long long>(M) * N;
+  const int nb = static_cast<int>(std::min<long long>(kSearchMaxBlocks, (count + kSearchThreads - 1) / kSearchThreads));
+  for (int i = 0; i < n_alpha; ++i) {
+    if ((st = awq_activation_scale(x, M, K, alphas[i], s, xs, stream)) != AWQ_OK) return st;
+    if ((st = awq_quantize_g128(W, s, N, K, qw, sc, zr, stream)) != AWQ_OK) return st;
+    if ((st = awq_w4a16_linear(xs, qw, sc, zr, y, M, N, K, stream)) != AWQ_OK) return st;
+    if ((st = launch_ex(awq_sq_error_kernel, dim3(nb, 1, 1), dim3(kSearchThreads, 1, 1), dim3(0, 0, 0), 0, cs, y_ref,
+                        reinterpret_cast<const __half*>(y), count, partial)) != AWQ_OK)
+      return st;
+    if ((st = launch_ex(awq_sq_error_final_kernel, dim3(1, 1, 1), dim3(32, 1, 1), dim3(0, 0, 0), 0, cs,
+                        static_cast<const double*>(partial), nb, err, i, i == n_alpha - 1 ? best : nullptr,
+                        n_alpha)) != AWQ_OK)
+      return st;
+  }
+  return AWQ_OK;
+}
+
+awq_status_t awq_w4a16_linear_qkv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                  const uint8_t* zeros, uint16_t* yq, uint16_t* yk, uint16_t* yv, int M, int Nq,
+                                  int Nkv, int K, awq_stream_t stream) {
+  if (!yk || !yv || Nq < 1 || Nkv < 1) return AWQ_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(Nq) + 2ll * Nkv;
+  if (N > kMaxRows) return AWQ_ERR_INVALID_ARG;
+  awq_status_t st = check_linear_args(x, qweight, scales, zeros, yq, M, static_cast<int>(N), K);
+  if (st != AWQ_OK) return st;
+  if (!aligned16(yk) || !aligned16(yv)) return AWQ_ERR_MISALIGNED;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != AWQ_OK) return st;
+  const EpiArgs epi = {reinterpret_cast<__half*>(yq), reinterpret_cast<__half*>(yk), reinterpret_cast<__half*>(yv),
+                       Nq, Nkv};
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const __half* sh = reinterpret_cast<const __half*>(scales);
+  if (M <= 32) return launch_gemv_epi<kEpiSplit3>(xh, qweight, sh, zeros, epi, M, static_cast<int>(N), K, dev, sms, cs);
+  return launch_gemm_epi<kEpiSplit3>(xh, qweight, sh, zeros, epi, M, static_cast<int>(N), K, dev, sms, cs);
+}
+
+awq_status_t awq_w4a16_linear_silu_mul(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
+                                       const uint8_t* zeros, uint16_t* h, int M, int I, int K, awq_stream_t stream) {
+  if (I < 16 || I % 16 != 0 || I > kMaxRows / 2) return AWQ_ERR_INVALID_ARG;
+  awq_status_t st = check_linear_args(x, qweight, scales, zeros, h, M, 2 * I, K);
+  if (st != AWQ_OK) return st;
+  int dev, sms;
+  if ((st = current_device(&dev, &sms)) != AWQ_OK) return st;
+  const EpiArgs epi = {reinterpret_cast<__half*>(h), nullptr, nullptr, 0, 0};
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const __half* sh = reinterpret_cast<const __half*>(scales);
+  if (M <= 32) return launch_gemv_epi<kEpiSiluMul>(xh, qweight, sh, zeros, epi, M, 2 * I, K, dev, sms, cs);
+  return launch_gemm_epi<kEpiSiluMul>(xh, qweight, sh, zeros, epi, M, 2 * I, K, dev, sms, cs);
 }
 
 awq_status_t awq_poll_device_status(awq_stream_t stream) {

@@ -22,7 +22,7 @@
 // (1.5*2^23 + 16, even, so ties go to even). Clamping: when every lane's
 // group keeps |w'/S| inside a 16-bit window (all groups of finite weights
 // whose range is above the 1e-5 floor), the low 16 bits of the rounded sum
-// are clamped as packed integers by two DPX instructions; otherwise
+// are clamped as packed integers by one DPX instruction; otherwise
 // clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z is taken in
 // fp32 before rounding (a clamped NaN becomes -z, i.e. code 0, as in the
 // IEEE form). Measured alternatives that were slower on B200 and are not
@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
   uint32_t phase = 0;
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int st = u / G, g = u % G;
-    if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget)) break;
+    // warp-uniform result: the shuffles below need the whole warp
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, s_abort, budget))) break;
     const uint8_t* sb = smem + stage * kQStageBytes;
     // ---- 64 weights of this lane: chunks c = 2i + half (16 B each), box c>>3, unit c&7 ^ (row & 7)
     uint4 raw[8];
@@ -250,8 +251,8 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
     // ---- codes: one quad (4 consecutive k = slots e0..e3) per (chunk i, step-half sb)
     uint32_t quad[8][2];
     // Packed-integer clamp: for |v| < 2^15 - 16 the low 16 bits of v + (1.5*2^23 + 16) are
-    // 16 + rint(v) (two's complement); one DPX add-max-relu and one min-relu on 16-bit pairs then
-    // give clamp(rint(v) + z, 0, 15). Every group of finite fp16 weights whose range is not the
+    // 16 + rint(v) (two's complement); one DPX add-min-relu on 16-bit pairs, max(min(a + b, 15), 0)
+    // with b = z - 16, then gives clamp(rint(v) + z, 0, 15). Every group of finite fp16 weights whose range is not the
     // 1e-5 floor has |v| <= 15 * 2^11 (range >= one fp16 ulp of max(|lo|, |hi|)); groups beyond
     // the 16-bit window (range at the floor, non-finite values) take the fp32 clamp below.
     const bool fast = fmaxf(fabsf(lo), fabsf(hi)) * rcp < 32000.0f;
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
             const uint64_t v2 = f2_fma(rho, rcp2, va);
             const float2 tq = f2_unpack(f2_add(v2, magic2));
             const uint32_t t16 = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x5410);
-            code2[pr] = __vimin_s16x2_relu(__viaddmax_s16x2_relu(t16, zoff2, 0u), 0x000F000Fu);
+            code2[pr] = __viaddmin_s16x2_relu(t16, zoff2, 0x000F000Fu);   // max(min(n + z, 15), 0)
           }
           quad[i][sbh] = __byte_perm(code2[0], code2[1], 0x6420);
         }
