@@ -152,13 +152,19 @@ AWQ_API awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scal
  * y = x . dequant^T with fp32 accumulation; dequant(q) = (q - z) * S.
  * Bitwise reproducible from call to call. Requires N >= 1, K >= 128,
  * K % 128 == 0.
- * Weight prefetch: the kernel starts reading qweight, scales and zeros as soon
- * as it is resident, which under programmatic dependent launch can be before
- * the preceding kernel of `stream` has finished (x and y are touched only
- * after it has). The packed weights must therefore be complete before that
- * preceding kernel begins: true when they were written by an earlier kernel or
- * copy, or by awq_quantize_g128, which lets no later kernel start before it
- * has completed and its writes are visible. */
+ * Weight prefetch and overlap: the kernel starts reading qweight, scales and
+ * zeros as soon as it is resident, and lets the next kernel of `stream` launch
+ * at once (programmatic dependent launch); x and y are touched only after the
+ * preceding kernel of `stream` has completed and its writes are visible. So a
+ * run of consecutive decode calls on one stream overlaps: each may start
+ * reading its weights while the earlier ones still run, back to the most
+ * recent stream operation that is not a decode call. The packed weights must
+ * be complete before that operation lets later work start: true for weights
+ * written by any earlier kernel or copy (ordinary kernels and copies let later
+ * work start only when they complete), and for awq_quantize_g128, which lets
+ * no later kernel start before its writes are visible. A kernel that writes
+ * packed weights must not trigger programmatic dependent launch before those
+ * writes. */
 AWQ_API awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
                             const uint8_t* zeros, uint16_t* y, int M, int N, int K,
                             awq_stream_t stream);

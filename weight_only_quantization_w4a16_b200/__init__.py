@@ -108,6 +108,9 @@ def _check(fn: str, status: int):
         raise AWQError(fn, status, status_string(status))
 
 
+LAYOUT_VERSION = 2   # the packed-weight layout this binding's size checks assume
+
+
 def layout_version() -> int:
     return int(load_library().awq_layout_version())
 

@@ -244,94 +244,13 @@ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
 #define AWQ_GEMV_CL 2
 #endif
 
-template <int MT, int NT, int CW, int D, int SB, int NACC = 2, bool kSumX = false>
-awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y,
-                             int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using Cfg = GemvCfg<MT, NT, CW, D, SB>;
-  static_assert(!kSumX || MT == 1, "activation sums are taken for tokens 0 and 1 only");
-  auto kernel = awq_gemv_kernel<MT, NT, CW, D, SB, NACC, kSumX>;
-  constexpr int kMaxSmem = 227 * 1024;
-  static std::atomic<uint64_t> smem_done{0};
-  awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
-  if (st != AWQ_OK) return st;
-  GemvArgs a = {};
-  a.qweight = reinterpret_cast<const uint8_t*>(qw);
-  a.scales = reinterpret_cast<const uint8_t*>(sc);
-  a.zeros = zr;
-  a.y = y;
-  a.M = M;
-  a.N = N;
-  a.ntiles = ceil_div(N, kTileRows);
-  a.g2 = ceil_div(K / kGroup, 2);
-  a.units = ceil_div(a.ntiles, NT);
-  const bool swz = M > 2;
-  a.x_swizzle = swz ? 1 : 0;
-  a.off_scales = Cfg::kCodes;
-  a.off_zeros = a.off_scales + Cfg::kScales;
-  a.off_x = round_up(a.off_zeros + Cfg::kZeros, swz ? 1024 : 128);
-  a.x_box_bytes = 4 * SB * M * 128;
-  a.stage_bytes = round_up(a.off_x + a.x_box_bytes, swz ? 1024 : 128);
-  CUtensorMap map;
-  st = make_x_map_decode(&map, x, M, K, 4 * SB, swz);
-  if (st != AWQ_OK) return st;
-  // clusters: CL CTAs each, about one CTA per SM, never more clusters than units
-  // CL CTAs per cluster, at most 32 workers (warps) per cluster: a unit's contributors then fit
-  // one warp's lanes in the reduction
-  int cl = AWQ_GEMV_CL;
-  while (cl > 1 && (a.units < cl || cl * CW > 32)) cl /= 2;
-  static_assert(CW <= 32, "warps per CTA");
-  int clusters = std::max(1, std::min(num_sms / cl, a.units));
-  // partial-sum records per warp: the most units one warp's item range touches
-  const long long Wc = static_cast<long long>(cl) * CW;
-  int R = 1;
-  for (int c = 0; c < clusters; ++c) {
-    const long long u0 = static_cast<long long>(c) * a.units / clusters;
-    const long long u1 = static_cast<long long>(c + 1) * a.units / clusters;
-    const long long L = (u1 - u0) * a.g2;
-    for (long long w = 0; w < Wc; ++w) {
-      const long long lo = w * L / Wc, hi = (w + 1) * L / Wc;
-      if (hi > lo) R = std::max(R, static_cast<int>((hi - 1) / a.g2 - lo / a.g2 + 1));
-    }
-  }
-  a.rec_per_warp = R;
-  const size_t smem = static_cast<size_t>(CW) * D * a.stage_bytes +
-                      static_cast<size_t>(CW) * R * NT * kTileRows * M * 4 + static_cast<size_t>(CW) * D * 8 + 16 + 1024;
-  if (smem > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
-  static ClusterOccCache cache;
-  const int fit = max_active_clusters(kernel, Cfg::kThreads, smem, cl, dev, cache);
-  if (fit < 1) return AWQ_ERR_UNSUPPORTED;
-  if (clusters > fit) {
-    // fewer clusters than SMs / CL can be resident at once: use what fits (recompute R)
-    clusters = fit;
-    R = 1;
-    for (int c = 0; c < clusters; ++c) {
-      const long long u0 = static_cast<long long>(c) * a.units / clusters;
-      const long long u1 = static_cast<long long>(c + 1) * a.units / clusters;
-      const long long L = (u1 - u0) * a.g2;
-      for (long long w = 0; w < Wc; ++w) {
-        const long long lo = w * L / Wc, hi = (w + 1) * L / Wc;
-        if (hi > lo) R = std::max(R, static_cast<int>((hi - 1) / a.g2 - lo / a.g2 + 1));
-      }
-    }
-    a.rec_per_warp = R;
-  }
-  a.clusters = clusters;
-  const size_t smem2 = static_cast<size_t>(CW) * D * a.stage_bytes +
-                       static_cast<size_t>(CW) * a.rec_per_warp * NT * kTileRows * M * 4 +
-                       static_cast<size_t>(CW) * D * 8 + 16 + 1024;
-  if (smem2 > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
-  return launch_ex(kernel, dim3(clusters * cl, 1, 1), dim3(Cfg::kThreads, 1, 1), dim3(cl, 1, 1), smem2, stream, map,
-                   a);
-}
-
-// The shared-ring decode form: CL-CTA clusters over 16-row units, each CTA a contiguous item range
-// streamed by one producer lane into S stages of up to SB group pairs; CW consumer warps.
-template <int MT, int CW, int S, int SB, int NACC = 4, bool kSumX = false, int EPI = kEpiPlain>
-awq_status_t launch_gemv_ring_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
-                                  const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using Cfg = GemvRingCfg<CW, SB>;
-  static_assert(!kSumX || MT == 1, "activation sums are taken for tokens 0 and 1 only");
-  auto kernel = awq_gemv_ring_kernel<MT, CW, S, SB, NACC, kSumX, EPI>;
+// The decode kernel: CL-CTA clusters over 16-row units, each CTA a contiguous item range streamed
+// by one producer lane into S stages of up to CW * SBW group pairs; CW consumer warps.
+template <int MT, int CW, int S, int SBW, bool kSwz, int EPI = kEpiPlain>
+awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  using Cfg = GemvCfg<CW, SBW, kSwz>;
+  auto kernel = awq_gemv_kernel<MT, CW, S, SBW, kSwz, EPI>;
   constexpr int kMaxSmem = 227 * 1024;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
@@ -347,19 +266,13 @@ awq_status_t launch_gemv_ring_cfg(const __half* x, const uint32_t* qw, const __h
   a.n1 = epi.n1;
   a.M = M;
   a.N = N;
-  a.ntiles = ceil_div(N, kTileRows);
   a.g2 = ceil_div(K / kGroup, 2);
-  a.units = EPI == kEpiSiluMul ? 2 * (N / 32) : a.ntiles;
+  a.units = EPI == kEpiSiluMul ? 2 * (N / 32) : ceil_div(N, kTileRows);
   const int upc = EPI == kEpiSiluMul ? 2 : 1;   // units per indivisible cluster share
-  const bool swz = M > 2;
-  a.x_swizzle = swz ? 1 : 0;
-  a.off_scales = Cfg::kCodes;
-  a.off_zeros = a.off_scales + Cfg::kScales;
-  a.off_x = round_up(a.off_zeros + Cfg::kZeros, swz ? 1024 : 128);
-  a.x_box_bytes = 4 * SB * M * 128;
-  a.stage_bytes = round_up(a.off_x + a.x_box_bytes, swz ? 1024 : 128);
+  a.x_box_bytes = 4 * Cfg::kSB * M * 128;
+  a.stage_bytes = round_up(Cfg::kOffX + a.x_box_bytes, Cfg::kAlignX);
   CUtensorMap map;
-  st = make_x_map_decode(&map, x, M, K, 4 * SB, swz);
+  st = make_x_map_decode(&map, x, M, K, 4 * Cfg::kSB, kSwz);
   if (st != AWQ_OK) return st;
   const int shares = a.units / upc;
   int cl = AWQ_GEMV_CL;
@@ -398,82 +311,52 @@ awq_status_t launch_gemv_ring_cfg(const __half* x, const uint32_t* qw, const __h
                    map, a);
 }
 
-// The ring form with a fused epilogue for any M <= 32 (the stage shrinks as the x' box grows).
+// Compile-time tuning of the decode kernel for M <= 2 (the decode shape of one sequence):
+// consumer warps, ring stages, group pairs per warp and stage.
+#ifndef AWQ_GEMV_CW
+#define AWQ_GEMV_CW 8
+#endif
+#ifndef AWQ_GEMV_S
+#define AWQ_GEMV_S 4
+#endif
+#ifndef AWQ_GEMV_SBW
+#define AWQ_GEMV_SBW 1
+#endif
+
+// Stage shapes per token count: the x' box grows with M, so larger M takes fewer group pairs per
+// stage and fewer stages, keeping shared memory near half an SM.
 template <int EPI>
 awq_status_t launch_gemv_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
   switch ((M + 7) / 8) {
     case 1:
       if (M <= 2)
-        return launch_gemv_ring_cfg<1, 8, 4, 8, 4, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-      return launch_gemv_ring_cfg<1, 8, 4, 4, 4, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-    case 2: return launch_gemv_ring_cfg<2, 4, 3, 4, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-    case 3: return launch_gemv_ring_cfg<3, 4, 3, 2, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-    default: return launch_gemv_ring_cfg<4, 4, 3, 2, 2, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+        return launch_gemv_cfg<1, AWQ_GEMV_CW, AWQ_GEMV_S, AWQ_GEMV_SBW, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev,
+                                                                                     num_sms, stream);
+      return launch_gemv_cfg<1, 4, 4, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    case 2: {
+      const awq_status_t st = launch_gemv_cfg<2, 4, 3, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      // very wide layers: fewer consumer warps (smaller per-warp records), shorter ring
+      return launch_gemv_cfg<2, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    }
+    case 3: {
+      const awq_status_t st = launch_gemv_cfg<3, 4, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      return launch_gemv_cfg<3, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    }
+    default: {
+      const awq_status_t st = launch_gemv_cfg<4, 4, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      return launch_gemv_cfg<4, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+    }
   }
 }
 
-// Compile-time tuning of the decode kernel per token tile: warps per CTA, ring stages per warp,
-// group pairs per stage, accumulator chains, and the M <= 2 form (codes as subnormals, zero
-// point through the activation sums).
-#ifndef AWQ_GEMV1_CW
-#define AWQ_GEMV1_CW 8
-#endif
-#ifndef AWQ_GEMV1_D
-#define AWQ_GEMV1_D 2
-#endif
-#ifndef AWQ_GEMV1_SB
-#define AWQ_GEMV1_SB 2
-#endif
-#ifndef AWQ_GEMV1_NACC
-#define AWQ_GEMV1_NACC 4
-#endif
-#ifndef AWQ_GEMV_SUMX
-#define AWQ_GEMV_SUMX 0
-#endif
-
-#ifndef AWQ_GEMV_KIND
-#define AWQ_GEMV_KIND 2
-#endif
-#ifndef AWQ_GEMVR_CW
-#define AWQ_GEMVR_CW 8
-#endif
-#ifndef AWQ_GEMVR_S
-#define AWQ_GEMVR_S 4
-#endif
-#ifndef AWQ_GEMVR_SB
-#define AWQ_GEMVR_SB 8
-#endif
-
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
                          int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  const int mt = (M + 7) / 8;
   const EpiArgs epi = {y, nullptr, nullptr, 0, 0};
-  switch (mt) {
-    case 1:
-      if (AWQ_GEMV_KIND == 2) {
-        if (AWQ_GEMV_SUMX && M <= 2)
-          return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, AWQ_GEMVR_S, AWQ_GEMVR_SB, AWQ_GEMV1_NACC, true>(
-              x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-        if (M <= 2)
-          return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, AWQ_GEMVR_S, AWQ_GEMVR_SB, AWQ_GEMV1_NACC>(
-              x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-        // 3 <= M <= 8: the x' box grows with M, so stages hold fewer group pairs
-        return launch_gemv_ring_cfg<1, AWQ_GEMVR_CW, 4, 4, AWQ_GEMV1_NACC>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
-                                                                            stream);
-      }
-      if (AWQ_GEMV_SUMX && M <= 2)
-        return launch_gemv_cfg<1, 1, AWQ_GEMV1_CW, AWQ_GEMV1_D, AWQ_GEMV1_SB, AWQ_GEMV1_NACC, true>(
-            x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-      if (M <= 2)
-        return launch_gemv_cfg<1, 1, AWQ_GEMV1_CW, AWQ_GEMV1_D, AWQ_GEMV1_SB, AWQ_GEMV1_NACC>(x, qw, sc, zr, y, M, N,
-                                                                                            K, dev, num_sms, stream);
-      // 3 <= M <= 8: the x' box grows with M, so stages hold one group pair
-      return launch_gemv_cfg<1, 1, 8, 2, 1, AWQ_GEMV1_NACC>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 2: return launch_gemv_cfg<2, 2, 4, 3, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    case 3: return launch_gemv_cfg<3, 2, 4, 2, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-    default: return launch_gemv_cfg<4, 2, 4, 2, 1>(x, qw, sc, zr, y, M, N, K, dev, num_sms, stream);
-  }
+  return launch_gemv_epi<kEpiPlain>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
@@ -736,7 +619,10 @@ awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const ui
 
 awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
                               uint16_t* y, int M, int N, int K, awq_stream_t stream) {
-  if (M >= 1 && M <= 32) return awq_w4a16_gemv(x, qweight, scales, zeros, y, M, N, K, stream);
+  if (M >= 1 && M <= 32) {
+    const awq_status_t st = awq_w4a16_gemv(x, qweight, scales, zeros, y, M, N, K, stream);
+    if (st != AWQ_ERR_UNSUPPORTED) return st;   // no decode shape fits: the prefill kernel serves any size
+  }
   return awq_w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream);
 }
 
