@@ -231,6 +231,32 @@ AWQ_API awq_status_t awq_search_alpha(const uint16_t* x, const uint16_t* W, int 
                                       const float* alphas, int n_alpha, double* err, int* best,
                                       void* workspace, size_t workspace_bytes, awq_stream_t stream);
 
+/* The scale search above for callers that cannot allocate device memory: code
+ * that runs inside a host program which owns all of the GPU's memory (a serving
+ * engine with a preallocated pool, a plugin that is handed no allocator), and
+ * code that must not call cudaMalloc/cudaFree because they synchronize the
+ * device and stall the other streams' work. The paper has no counterpart; this
+ * is a library convenience. Arguments, results and status codes are those of
+ * awq_search_alpha, and so are the errors, bit for bit; the workspace is
+ * instead a fixed array of AWQ_SEARCH_NOALLOC_SCRATCH_BYTES (64 MiB) in the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits. Nothing here calls cudaMalloc, cudaFree or any
+ * allocating library routine.
+ *   Limit: awq_search_workspace_bytes(M, N, K) <= AWQ_SEARCH_NOALLOC_SCRATCH_BYTES
+ *   (e.g. a 4096 x 4096 layer with up to 1781 calibration rows, 8192 x 8192 with
+ *   up to 491); larger shapes return AWQ_ERR_INVALID_ARG and launch nothing.
+ *   Set-up: the first call on a device, with that device current, looks up the
+ *   array's device address; make that first call before any stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps the last
+ *   call's contents (no byte of it needs to start at zero: each call writes
+ *   everything it reads). Calls whose work can overlap on the GPU (streams not
+ *   ordered with each other) race on the array and give undefined errors:
+ *   order them on one stream or with events. */
+#define AWQ_SEARCH_NOALLOC_SCRATCH_BYTES (64u << 20)
+AWQ_API awq_status_t awq_search_alpha_noalloc(const uint16_t* x, const uint16_t* W, int M, int N, int K,
+                                              const float* alphas, int n_alpha, double* err, int* best,
+                                              awq_stream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the device status word of the
  * current device. Returns AWQ_ERR_TIMEOUT if a kernel since the last poll gave
  * up a bounded wait (its outputs are then undefined), AWQ_ERR_CUDA if the

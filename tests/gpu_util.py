@@ -27,7 +27,7 @@ def lib():
 
 
 def oracle_packed(W: np.ndarray, s):
-    """Oracle codes for W (folded with s) packed to layout v1 (numpy arrays)."""
+    """Oracle codes for W (folded with s) packed to layout v2 (numpy arrays)."""
     q, S, z = O.quantize_groups(O.fold_weights(W, s))
     return O.pack(q, S, z), (q, S, z)
 

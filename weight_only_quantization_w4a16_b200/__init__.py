@@ -70,6 +70,7 @@ _SIGS = {
     "awq_w4a16_linear_qkv": ([_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _VP], _I),
     "awq_w4a16_linear_silu_mul": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_search_alpha": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _VP, ctypes.c_size_t, _VP], _I),
+    "awq_search_alpha_noalloc": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _VP], _I),
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
     "awq_debug_drop_first_copy": ([_I], _I),
 }
@@ -362,6 +363,38 @@ def awq_search_alpha(x, W, alphas=None, workspace=None):
     st = lib.awq_search_alpha(_ptr(x), _ptr(W), M, N, K, ctypes.cast(a, _VP), len(alphas), _ptr(err), _ptr(best),
                               _ptr(workspace), workspace.numel(), _stream_ptr())
     _check("awq_search_alpha", st)
+    return err, best, list(alphas)
+
+
+SEARCH_NOALLOC_SCRATCH_BYTES = 64 << 20   # the fixed scratch of awq_search_alpha_noalloc
+
+
+def awq_search_alpha_noalloc(x, W, alphas=None):
+    """The scale search on the library's fixed device scratch (no workspace argument).
+
+    For callers that cannot allocate device memory themselves; results equal awq_search_alpha's.
+    Shapes whose workspace would exceed SEARCH_NOALLOC_SCRATCH_BYTES raise ValueError. Only the
+    outputs err and best are allocated here, by the caller's framework.
+    """
+    torch = _torch()
+    _need(x, torch.float16, "x", 2)
+    _need(W, torch.float16, "W", 2)
+    M, K = x.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError(f"W must have K={K} columns")
+    if alphas is None:
+        alphas = [i / 20.0 for i in range(20)]
+    a = (ctypes.c_float * len(alphas))(*[float(v) for v in alphas])
+    lib = load_library()
+    need = int(lib.awq_search_workspace_bytes(M, N, K))
+    if need == 0 or need > SEARCH_NOALLOC_SCRATCH_BYTES:
+        raise ValueError(f"shape out of range for the search without workspace ({need} bytes needed)")
+    err = torch.empty(len(alphas), dtype=torch.float64, device=x.device)
+    best = torch.empty(1, dtype=torch.int32, device=x.device)
+    st = lib.awq_search_alpha_noalloc(_ptr(x), _ptr(W), M, N, K, ctypes.cast(a, _VP), len(alphas), _ptr(err),
+                                      _ptr(best), _stream_ptr())
+    _check("awq_search_alpha_noalloc", st)
     return err, best, list(alphas)
 
 

@@ -479,6 +479,33 @@ inline bool search_shape_ok(int M, int N, int K) {
          static_cast<long long>(M) * K <= (1ll << 31) - 1 && static_cast<long long>(M) * N <= (1ll << 31) - 1;
 }
 
+
+// Scratch of awq_search_alpha_noalloc: a file-scope device array, so that callers which cannot
+// allocate device memory can still run the search. Every device on which this library's kernels
+// are loaded holds it until the process exits. In host code `g_search_scratch` only names the
+// symbol; its address on a device comes from cudaGetSymbolAddress with that device current.
+static __device__ __align__(256) unsigned char g_search_scratch[AWQ_SEARCH_NOALLOC_SCRATCH_BYTES];
+std::atomic<void*> g_search_scratch_ptr[kMaxDevices];
+std::mutex g_search_scratch_mutex;
+
+// Device address of g_search_scratch on `dev` (the current device), looked up once per device.
+awq_status_t search_scratch(int dev, void** out) {
+  void* p = g_search_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_search_scratch_mutex);
+    p = g_search_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      if (cudaGetSymbolAddress(&p, g_search_scratch) != cudaSuccess || p == nullptr) {
+        (void)cudaGetLastError();
+        return AWQ_ERR_CUDA;
+      }
+      g_search_scratch_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return AWQ_OK;
+}
+
 }  // namespace
 }  // namespace awq
 
@@ -676,6 +703,19 @@ awq_status_t awq_search_alpha(const uint16_t* x, const uint16_t* W, int M, int N
       return st;
   }
   return AWQ_OK;
+}
+
+awq_status_t awq_search_alpha_noalloc(const uint16_t* x, const uint16_t* W, int M, int N, int K, const float* alphas,
+                                      int n_alpha, double* err, int* best, awq_stream_t stream) {
+  if (!search_shape_ok(M, N, K) || search_ws(M, N, K).total > static_cast<size_t>(AWQ_SEARCH_NOALLOC_SCRATCH_BYTES))
+    return AWQ_ERR_INVALID_ARG;
+  int dev, sms;
+  awq_status_t st = current_device(&dev, &sms);
+  if (st != AWQ_OK) return st;
+  void* scratch = nullptr;
+  if ((st = search_scratch(dev, &scratch)) != AWQ_OK) return st;
+  return awq_search_alpha(x, W, M, N, K, alphas, n_alpha, err, best, scratch,
+                          static_cast<size_t>(AWQ_SEARCH_NOALLOC_SCRATCH_BYTES), stream);
 }
 
 awq_status_t awq_w4a16_linear_qkv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales,
