@@ -44,9 +44,12 @@
 namespace awq {
 
 // ------------------------------------------------------------------------------------
-// Cluster barrier (all 32 lanes of a warp execute it together).
+// Cluster barrier, split into arrive and wait (all 32 lanes of a warp execute each together).
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -81,16 +84,18 @@ struct GemvCfg {
 };
 
 // Loads the B fragments (x') of one 64-k tile for the lane's token rows: 32 bytes per 8-token
-// tile (chunks 2t and 2t+1 of row kt_local*M + m of the x' box), zero for tokens >= M.
+// tile (chunks 2t and 2t+1 of row kt_local*M + m of the x' box). With one token tile, lanes of
+// tokens m >= M read token M-1 instead: those MMA columns are never stored, so they need no
+// zeroing. (With more tiles the select keeps register pressure lower.)
 template <int MT, bool kSwz>
 __device__ __forceinline__ void gemv_load_x(uint4 (&xv)[MT][2], const uint8_t* xs, int kt_local, int M, int r, int t) {
 #pragma unroll
   for (int j = 0; j < MT; ++j) {
-    const int m = 8 * j + r;
+    const int m = MT == 1 ? min(r, M - 1) : 8 * j + r;
     const int row = kt_local * M + m;
     const int c0 = kSwz ? ((2 * t) ^ (row & 7)) : 2 * t;
     const int c1 = kSwz ? ((2 * t + 1) ^ (row & 7)) : 2 * t + 1;
-    const bool live = m < M;
+    const bool live = MT == 1 || m < M;
     xv[j][0] = live ? *reinterpret_cast<const uint4*>(xs + row * 128 + c0 * 16) : make_uint4(0, 0, 0, 0);
     xv[j][1] = live ? *reinterpret_cast<const uint4*>(xs + row * 128 + c1 * 16) : make_uint4(0, 0, 0, 0);
   }
@@ -142,9 +147,11 @@ __device__ __forceinline__ void gemv_group(float (&acc)[MT][4], const uint4& c0,
 }
 
 // MT: 8-token tiles (M <= 8 MT); CW: consumer warps; S: ring stages; SBW: group pairs per consumer
-// warp and stage; kSwz: the x' box uses the 128-byte swizzle (M > 2); EPI: epilogue.
-template <int MT, int CW, int S, int SBW, bool kSwz, int EPI>
-__global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, 1)
+// warp and stage; kSwz: the x' box uses the 128-byte swizzle (M > 2); EPI: epilogue; MINB: CTAs
+// per SM the registers must allow (2 lets the next decode launch's CTAs become resident, and
+// prefetch their weights, while this one runs).
+template <int MT, int CW, int S, int SBW, bool kSwz, int EPI, int MINB>
+__global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, MINB)
     awq_gemv_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemvArgs a) {
   using C = GemvCfg<CW, SBW, kSwz>;
   constexpr int SB = C::kSB;
@@ -161,7 +168,8 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, 1)
   const int rec_elems = 16 * M;   // floats per record (one 16-row unit)
   const int R = a.rec_per_warp;
   float* rec_all = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * a.stage_bytes);   // [CW][R][16][M]
-  uint64_t* full = reinterpret_cast<uint64_t*>(rec_all + static_cast<size_t>(CW) * R * rec_elems);
+  float* recv = rec_all + static_cast<size_t>(CW) * R * rec_elems;   // [2][16][M]: partials pushed by rank 1
+  uint64_t* full = reinterpret_cast<uint64_t*>(recv + 2 * rec_elems);
   uint64_t* empty = full + S;
   volatile int* s_abort = reinterpret_cast<volatile int*>(empty + S);
 
@@ -186,6 +194,7 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
+  if (CL == 2) cluster_arrive_relaxed();   // first cluster phase: this CTA has started
   // The next kernel of the stream may launch at once: it reads only its own packed weights before
   // its griddepcontrol.wait, which returns after this grid has completed.
   pdl_launch_dependents();
@@ -316,64 +325,67 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, 1)
     if (ok && i0 < i1) flush();
   }
 
-  // ---- the CTA adds its consumer warps' records, in warp order (all threads of the CTA)
+  // ---- epilogue. The cluster's items are split at L/2 between its two CTAs, so at most one
+  // block of units (one unit; one gate/up unit pair with kEpiSiluMul) is shared. Each CTA adds its
+  // consumer warps' records in warp order and stores the blocks it holds alone; for the shared
+  // block, rank 1 pushes its sums into rank 0's shared memory, and rank 0 adds them after its own
+  // (rank order: deterministic, no global scratch, no atomics).
   __syncthreads();
-  if (*s_abort == 0) {
-    const int n_rec = (i0 < i1) ? (i1 - 1) / G2 - i0 / G2 + 1 : 0;
-    for (int e = threadIdx.x; e < n_rec * rec_elems; e += blockDim.x) {
-      float v = 0.f;
-      for (int w = 0; w < CW; ++w) v += rec_all[static_cast<size_t>(w) * R * rec_elems + e];
-      rec_all[e] = v;   // warp 0's records now hold the CTA's sums
-    }
-  }
-  // ---- cluster reduction: each output is the sum of the records of the CTAs that touched its
-  // unit, in rank order. One warp per unit (per gate/up pair with kEpiSiluMul).
-  cluster_arrive();
-  cluster_wait();
-  if (*s_abort == 0) {
-    const uint32_t Lu = static_cast<uint32_t>(L), CLu = static_cast<uint32_t>(CL);
-    const int nunits = u1 - u0;
-    const int nwarps = CW + 1;
-    // the sum over the contributing CTAs of element (row, m) of relative unit ur
-    auto unit_sum = [&](int ur, int row, int m) -> float {
-      const uint32_t first = static_cast<uint32_t>(ur) * G2, last = first + G2 - 1;
-      const uint32_t cf = ((first + 1) * CLu - 1) / Lu, cl_ = ((last + 1) * CLu - 1) / Lu;
-      float v = 0.f;
-      for (uint32_t c = cf; c <= cl_; ++c) {
-        const uint32_t ac = c * Lu / CLu, bc = (c + 1) * Lu / CLu;
-        if (bc == ac) continue;
-        const int rr = ur - static_cast<int>(ac / G2);
-        v += cluster.map_shared_rank(rec_all, static_cast<int>(c))[rr * rec_elems + row * M + m];
-      }
-      return v;
-    };
+  const int bsz = upc * G2;                                  // items per block
+  const int split = L / 2;
+  const bool shared_blk = CL == 2 && split > 0 && split < L && (split - 1) / bsz == split / bsz;
+  const int bb = split / bsz;                                // the shared block (relative)
+  const bool live = *s_abort == 0 && i0 < i1;
+  const int uf = i0 / G2, ul = (i1 - 1) / G2;                // units of this CTA's records (relative)
+  // element e of relative unit ur summed over this CTA's warps (zero for a unit it did not touch)
+  auto cta_sum = [&](int ur, int e) -> float {
+    if (ur < uf || ur > ul) return 0.f;
+    const float* pr = rec_all + static_cast<size_t>(ur - uf) * rec_elems + e;
+    float v = 0.f;
+#pragma unroll 4
+    for (int w = 0; w < CW; ++w) v += pr[static_cast<size_t>(w) * R * rec_elems];
+    return v;
+  };
+  // stores block b; `extra` (rank 0, shared block) holds rank 1's sums of the block's units
+  auto finalize = [&](int b, int e, const float* extra) {
+    const int row = e / M, m = e - row * M;
     if (EPI == kEpiSiluMul) {
+      float g = cta_sum(2 * b, e), u = cta_sum(2 * b + 1, e);
+      if (extra != nullptr) { g += extra[e]; u += extra[rec_elems + e]; }
       const int I = a.N / 2;
-      for (int pr = rank * nwarps + warp; 2 * pr < nunits; pr += CL * nwarps) {
-        const int j = u0 / 2 + pr;   // gate tile j, up tile P + j
-        for (int e = lane; e < rec_elems; e += 32) {
-          const int row = e / M, m = e - row * M;
-          const float g = unit_sum(2 * pr, row, m), u = unit_sum(2 * pr + 1, row, m);
-          const int i = 16 * j + row;
-          if (i < I) a.y[static_cast<size_t>(m) * I + i] = __float2half_rn(silu_mul(g, u));
-        }
-      }
+      const int i = 16 * (u0 / 2 + b) + row;
+      if (i < I) a.y[static_cast<size_t>(m) * I + i] = __float2half_rn(silu_mul(g, u));
     } else {
-      const EpiArgs epi = {a.y, a.y1, a.y2, a.n0, a.n1};
-      for (int ur = rank * nwarps + warp; ur < nunits; ur += CL * nwarps) {
-        const long long nbase = static_cast<long long>(u0 + ur) * 16;
-        for (int e = lane; e < rec_elems; e += 32) {
-          const int row = e / M, m = e - row * M;
-          const float v = unit_sum(ur, row, m);
-          const long long n = nbase + row;
-          if (n < a.N) epi_store<EPI>(epi, m, n, a.N, v);
-        }
+      float v = cta_sum(b, e);
+      if (extra != nullptr) v += extra[e];
+      const long long n = static_cast<long long>(u0 + b) * 16 + row;
+      if (n < a.N) epi_store<EPI>(EpiArgs{a.y, a.y1, a.y2, a.n0, a.n1}, m, n, a.N, v);
+    }
+  };
+  if (CL == 2) {
+    cluster_wait();                                          // both CTAs have started
+    if (rank == 0) cluster_arrive_relaxed();                 // second phase: rank 0 only receives
+    else {
+      if (live && shared_blk) {
+        float* dst = cluster.map_shared_rank(recv, 0);
+        for (int idx = threadIdx.x; idx < upc * rec_elems; idx += blockDim.x)
+          dst[idx] = cta_sum(bb * upc + idx / rec_elems, idx % rec_elems);
       }
+      cluster_arrive();                                      // release: the pushed sums
     }
   }
-  // no CTA leaves while another may still read its shared memory
-  cluster_arrive();
-  cluster_wait();
+  if (live) {
+    const int fb = uf / upc, lb = ul / upc;
+    const int b0 = (shared_blk && rank == 1) ? fb + 1 : fb;  // rank 1's first block is the shared one
+    const int b1 = (shared_blk && rank == 0) ? lb - 1 : lb;  // rank 0's last block is the shared one
+    for (int idx = threadIdx.x; idx < (b1 - b0 + 1) * rec_elems; idx += blockDim.x)
+      finalize(b0 + idx / rec_elems, idx % rec_elems, nullptr);
+  }
+  if (CL == 2) {
+    cluster_wait();                                          // rank 1's sums are in `recv`
+    if (rank == 0 && live && shared_blk)
+      for (int e = threadIdx.x; e < rec_elems; e += blockDim.x) finalize(bb, e, recv);
+  }
 }
 
 }  // namespace awq

@@ -243,14 +243,15 @@ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
 #ifndef AWQ_GEMV_CL
 #define AWQ_GEMV_CL 2
 #endif
+static_assert(AWQ_GEMV_CL == 1 || AWQ_GEMV_CL == 2, "the decode epilogue shares blocks between at most two CTAs");
 
 // The decode kernel: CL-CTA clusters over 16-row units, each CTA a contiguous item range streamed
 // by one producer lane into S stages of up to CW * SBW group pairs; CW consumer warps.
-template <int MT, int CW, int S, int SBW, bool kSwz, int EPI = kEpiPlain>
+template <int MT, int CW, int S, int SBW, bool kSwz, int EPI = kEpiPlain, int MINB = 1>
 awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
   using Cfg = GemvCfg<CW, SBW, kSwz>;
-  auto kernel = awq_gemv_kernel<MT, CW, S, SBW, kSwz, EPI>;
+  auto kernel = awq_gemv_kernel<MT, CW, S, SBW, kSwz, EPI, MINB>;
   constexpr int kMaxSmem = 227 * 1024;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, kMaxSmem, dev, smem_done);
@@ -293,7 +294,7 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
   };
   auto smem_of = [&](int R) {
     return static_cast<size_t>(S) * a.stage_bytes + static_cast<size_t>(CW) * R * kTileRows * M * 4 +
-           static_cast<size_t>(2 * S) * 8 + 16 + 1024;
+           static_cast<size_t>(2) * kTileRows * M * 4 + static_cast<size_t>(2 * S) * 8 + 16 + 1024;
   };
   int R = records(clusters);
   if (smem_of(R) > static_cast<size_t>(kMaxSmem)) return AWQ_ERR_UNSUPPORTED;
@@ -312,15 +313,18 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
 }
 
 // Compile-time tuning of the decode kernel for M <= 2 (the decode shape of one sequence):
-// consumer warps, ring stages, group pairs per warp and stage.
+// consumer warps, ring stages, group pairs per warp and stage, CTAs per SM the registers allow.
 #ifndef AWQ_GEMV_CW
 #define AWQ_GEMV_CW 8
 #endif
 #ifndef AWQ_GEMV_S
-#define AWQ_GEMV_S 4
+#define AWQ_GEMV_S 2
 #endif
 #ifndef AWQ_GEMV_SBW
-#define AWQ_GEMV_SBW 1
+#define AWQ_GEMV_SBW 2
+#endif
+#ifndef AWQ_GEMV_MINB
+#define AWQ_GEMV_MINB 2
 #endif
 
 // Stage shapes per token count: the x' box grows with M, so larger M takes fewer group pairs per
@@ -331,8 +335,8 @@ awq_status_t launch_gemv_epi(const __half* x, const uint32_t* qw, const __half* 
   switch ((M + 7) / 8) {
     case 1:
       if (M <= 2)
-        return launch_gemv_cfg<1, AWQ_GEMV_CW, AWQ_GEMV_S, AWQ_GEMV_SBW, false, EPI>(x, qw, sc, zr, epi, M, N, K, dev,
-                                                                                     num_sms, stream);
+        return launch_gemv_cfg<1, AWQ_GEMV_CW, AWQ_GEMV_S, AWQ_GEMV_SBW, false, EPI, AWQ_GEMV_MINB>(
+            x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
       return launch_gemv_cfg<1, 4, 4, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
     case 2: {
       const awq_status_t st = launch_gemv_cfg<2, 4, 3, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
