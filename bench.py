@@ -646,6 +646,9 @@ def sub_records(torch, P, timer, dev, l2, hbm_peak, tc_peak, tc_sus, peak_src, w
     ba = bytes_act_scale(4096, 4096)
     out["act_scale"] = {"kernel": "awq_act_scale_kernel", "bound": "hbm", "shape": "M=4096, K=4096", "us": us,
                         "GBps": ba / us / 1e3, "frac": ba / us / 1e3 / hbm_peak, "peak": hbm_peak}
+    # decode kernel vs prefill kernel on the batched-decode shapes, and what awq_w4a16_linear picks
+    if M == 1 and wl.name == "llama2_7b_decode_m1":
+        out["crossover"] = crossover(torch, P, timer, dev, l2)
     # a dependent decode chain of one Llama-2-7B block at M = 1: scale -> fused q/k/v (split) ->
     # scale -> o_proj -> scale -> fused gate+up (SiLU * up) -> scale -> down, each layer fed by the
     # previous output (q stands in for the attention output), weights rotated through >= 4x L2
@@ -667,6 +670,37 @@ def sub_records(torch, P, timer, dev, l2, hbm_peak, tc_peak, tc_sus, peak_src, w
                             "note": "activation statistic + fold/quantize + decode GEMV for every layer of the "
                                     "workload (fp16 weights re-quantized every step)"}
     return out
+
+
+def crossover(torch, P, timer, dev, l2, Ms=(4, 8, 16, 32)):
+    """µs per launch of the decode kernel, the prefill kernel and the dispatching call per layer and M."""
+    wl3 = workloads.WORKLOADS["llama2_7b_decode_batched"]
+    recs = []
+    for li, layer in enumerate(wl3.layers):
+        x, W = workloads.layer_inputs(wl3, li, max(Ms))
+        N, K = layer.N, layer.K
+        with torch.cuda.stream(timer.stream):
+            s, xs = P.awq_activation_scale(torch.from_numpy(x).to(dev), 0.5)
+            Wd = torch.from_numpy(W).to(dev)
+            packed = P.awq_quantize_g128(Wd, s)
+            del Wd
+            nset = rotation_sets(packed_bytes(N, K), l2)
+            copies = [packed] + [tuple(t.clone() for t in packed) for _ in range(nset - 1)]
+            for Mx in Ms:
+                xm = xs[:Mx].contiguous()
+                y = torch.empty((Mx, N), dtype=torch.float16, device=dev)
+                r = {"layer": f"{wl3.name}/{N}x{K}", "M": Mx}
+                for name, fn in (("gemv", P.awq_w4a16_gemv), ("gemm", P.awq_w4a16_gemm), ("linear", P.awq_w4a16_linear)):
+                    us, g = per_launch_us(timer, lambda i, fn=fn: fn(xm, *copies[i % nset], N, y), launches=16)
+                    del g
+                    r[name + "_us"] = us
+                r["faster"] = "gemv" if r["gemv_us"] <= r["gemm_us"] else "gemm"
+                recs.append(r)
+            del copies
+    return {"records": recs,
+            "note": "16 launches back to back in a CUDA graph over packed copies rotated through >= 4x L2, median "
+                    "of 5; awq_w4a16_linear takes the decode kernel for M <= 32 unless its full-size configuration "
+                    "does not fit in shared memory"}
 
 
 def decode_layer_chain(torch, P, timer, dev, l2, hbm_peak, wl):

@@ -328,10 +328,15 @@ awq_status_t launch_gemv_cfg(const __half* x, const uint32_t* qw, const __half* 
 #endif
 
 // Stage shapes per token count: the x' box grows with M, so larger M takes fewer group pairs per
-// stage and fewer stages, keeping shared memory near half an SM.
+// stage and fewer stages, keeping shared memory near half an SM. For very wide layers at M > 8 the
+// per-warp records outgrow shared memory and only a smaller configuration (fewer consumer warps,
+// shorter ring) fits; with `fallback` false that case returns AWQ_ERR_UNSUPPORTED instead, so that
+// the layer-level dispatch can take the prefill kernel, which measures faster there (M = 32 on the
+// 22016- and 28672-row layers).
 template <int EPI>
 awq_status_t launch_gemv_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
-                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream,
+                             bool fallback = true) {
   switch ((M + 7) / 8) {
     case 1:
       if (M <= 2)
@@ -340,27 +345,27 @@ awq_status_t launch_gemv_epi(const __half* x, const uint32_t* qw, const __half* 
       return launch_gemv_cfg<1, 4, 4, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
     case 2: {
       const awq_status_t st = launch_gemv_cfg<2, 4, 3, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      if (st != AWQ_ERR_UNSUPPORTED || !fallback) return st;
       // very wide layers: fewer consumer warps (smaller per-warp records), shorter ring
       return launch_gemv_cfg<2, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
     }
     case 3: {
       const awq_status_t st = launch_gemv_cfg<3, 4, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      if (st != AWQ_ERR_UNSUPPORTED || !fallback) return st;
       return launch_gemv_cfg<3, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
     }
     default: {
       const awq_status_t st = launch_gemv_cfg<4, 4, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-      if (st != AWQ_ERR_UNSUPPORTED) return st;
+      if (st != AWQ_ERR_UNSUPPORTED || !fallback) return st;
       return launch_gemv_cfg<4, 2, 2, 1, true, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
     }
   }
 }
 
 awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
-                         int N, int K, int dev, int num_sms, cudaStream_t stream) {
+                         int N, int K, int dev, int num_sms, cudaStream_t stream, bool fallback = true) {
   const EpiArgs epi = {y, nullptr, nullptr, 0, 0};
-  return launch_gemv_epi<kEpiPlain>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+  return launch_gemv_epi<kEpiPlain>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream, fallback);
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
@@ -650,9 +655,16 @@ awq_status_t awq_w4a16_gemm(const uint16_t* x, const uint32_t* qweight, const ui
 
 awq_status_t awq_w4a16_linear(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,
                               uint16_t* y, int M, int N, int K, awq_stream_t stream) {
+  // M <= 32: the decode kernel in its primary configuration, which measures faster than the
+  // prefill kernel at every such M on the Llama-2 7B/70B shapes; otherwise the prefill kernel.
   if (M >= 1 && M <= 32) {
-    const awq_status_t st = awq_w4a16_gemv(x, qweight, scales, zeros, y, M, N, K, stream);
-    if (st != AWQ_ERR_UNSUPPORTED) return st;   // no decode shape fits: the prefill kernel serves any size
+    awq_status_t st = check_linear_args(x, qweight, scales, zeros, y, M, N, K);
+    if (st != AWQ_OK) return st;
+    int dev, sms;
+    if ((st = current_device(&dev, &sms)) != AWQ_OK) return st;
+    st = launch_gemv(reinterpret_cast<const __half*>(x), qweight, reinterpret_cast<const __half*>(scales), zeros,
+                     reinterpret_cast<__half*>(y), M, N, K, dev, sms, reinterpret_cast<cudaStream_t>(stream), false);
+    if (st != AWQ_ERR_UNSUPPORTED) return st;
   }
   return awq_w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream);
 }
@@ -738,7 +750,10 @@ awq_status_t awq_w4a16_linear_qkv(const uint16_t* x, const uint32_t* qweight, co
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const __half* xh = reinterpret_cast<const __half*>(x);
   const __half* sh = reinterpret_cast<const __half*>(scales);
-  if (M <= 32) return launch_gemv_epi<kEpiSplit3>(xh, qweight, sh, zeros, epi, M, static_cast<int>(N), K, dev, sms, cs);
+  if (M <= 32) {
+    st = launch_gemv_epi<kEpiSplit3>(xh, qweight, sh, zeros, epi, M, static_cast<int>(N), K, dev, sms, cs, false);
+    if (st != AWQ_ERR_UNSUPPORTED) return st;
+  }
   return launch_gemm_epi<kEpiSplit3>(xh, qweight, sh, zeros, epi, M, static_cast<int>(N), K, dev, sms, cs);
 }
 
@@ -753,7 +768,10 @@ awq_status_t awq_w4a16_linear_silu_mul(const uint16_t* x, const uint32_t* qweigh
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const __half* xh = reinterpret_cast<const __half*>(x);
   const __half* sh = reinterpret_cast<const __half*>(scales);
-  if (M <= 32) return launch_gemv_epi<kEpiSiluMul>(xh, qweight, sh, zeros, epi, M, 2 * I, K, dev, sms, cs);
+  if (M <= 32) {
+    st = launch_gemv_epi<kEpiSiluMul>(xh, qweight, sh, zeros, epi, M, 2 * I, K, dev, sms, cs, false);
+    if (st != AWQ_ERR_UNSUPPORTED) return st;
+  }
   return launch_gemm_epi<kEpiSiluMul>(xh, qweight, sh, zeros, epi, M, 2 * I, K, dev, sms, cs);
 }
 
