@@ -64,6 +64,10 @@ def parse_args(argv=None):
     p.add_argument("--no-sub", action="store_true", help="skip the sub-records")
     p.add_argument("--reference-budget-s", type=float, default=150.0,
                    help="CPU seconds the reference (oracle) arm may spend in total")
+    p.add_argument("--profile-kernel", choices=["gemv", "gemm", "quantize", "act_scale"], default=None,
+                   help="only run --launches launches of one kernel on layer --layer of the workload (for ncu)")
+    p.add_argument("--layer", type=int, default=0)
+    p.add_argument("--launches", type=int, default=4)
     return p.parse_args(argv)
 
 
@@ -784,8 +788,41 @@ def end_to_end(torch, P, stream, host, L, M, steps, world, decode):
                     "kernel) with pinned-host x copied in and y copied out every step; packed weights resident"}
 
 
+def profile_kernel(args):
+    """A few launches of one kernel on one layer of a workload, inputs prepared beforehand: the small,
+    self-contained case an ncu capture of that kernel runs on."""
+    import torch
+    import weight_only_quantization_w4a16_b200 as P
+    P.load_library()
+    torch.cuda.set_device(0)
+    wl = workloads.WORKLOADS[args.workload]
+    M = args.m if args.m is not None else wl.Ms[0]
+    layer = wl.layers[args.layer]
+    x, W = workloads.layer_inputs(wl, args.layer, M)
+    xd, Wd = torch.from_numpy(x).cuda(), torch.from_numpy(W).cuda()
+    s, xs = P.awq_activation_scale(xd, 0.5)
+    packed = P.awq_quantize_g128(Wd, s)
+    y = torch.empty((M, layer.N), dtype=torch.float16, device="cuda")
+    for _ in range(args.launches):
+        if args.profile_kernel == "gemv":
+            P.awq_w4a16_gemv(xs, *packed, layer.N, y)
+        elif args.profile_kernel == "gemm":
+            P.awq_w4a16_gemm(xs, *packed, layer.N, y)
+        elif args.profile_kernel == "quantize":
+            P.awq_quantize_g128(Wd, s, packed)
+        else:
+            P.awq_activation_scale(xd, 0.5, s, xs)
+    torch.cuda.synchronize()
+    assert P.awq_poll_device_status() == P.AWQ_OK
+    print(f"{args.profile_kernel}: {args.launches} launches on {wl.name} layer {args.layer} "
+          f"({layer.N}x{layer.K}), M = {M}", flush=True)
+
+
 def main():
     args = parse_args()
+    if args.profile_kernel:
+        profile_kernel(args)
+        return
     world, rank, local = dist_init(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
