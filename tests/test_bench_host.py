@@ -20,11 +20,12 @@ def test_code_hash_ignores_comments_and_whitespace_only():
 def test_traffic_record_applies_only_to_its_workload_and_unchanged_code():
     d = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
     wl, M = d["_workload"], d["_M"]
+    assert "awq_gemv.cuh" in d   # the kernel of the default bench step
     for name in ("awq_quant.cuh", "awq_gemv.cuh", "awq_act.cuh"):
         # reported exactly while the recorded code hash matches the kernel code
         e = bench.profile_traffic(name, wl, M)
-        if d[name]["source_sha256_16"] == bench.kernel_source_hash(name):
-            assert e is not None and e["bytes_per_launch"] > 0
+        if name in d and d[name]["source_sha256_16"] == bench.kernel_source_hash(name):
+            assert e is not None and e["bytes_per_step"] > 0
         else:
             assert e is None
         # another workload or M never gets a traffic figure
