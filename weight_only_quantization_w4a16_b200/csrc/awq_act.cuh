@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kActThreads) awq_act_scale_kernel(const __half
   __shared__ uint64_t s_csum[kActCols];
   __shared__ float s_scale[kActCols];
 
-  pdl_enter();
+  pdl_enter_early();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k0 = blockIdx.x * kActCols;
   const int rsub = lane >> 3;         // 0..3: row within the warp's 4-row step
@@ -146,7 +146,7 @@ constexpr int kActSmallMaxM = 32;
 __global__ void __launch_bounds__(128) awq_act_scale_small_kernel(const __half* __restrict__ x, int M, int K,
                                                              float alpha, float* __restrict__ s_out,
                                                              __half* __restrict__ x_scaled) {
-  pdl_enter();
+  pdl_enter_early();
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= K) return;
   const unsigned short* xb = reinterpret_cast<const unsigned short*>(x);
@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(128) awq_act_scale_small_kernel(const __half* 
 __global__ void __launch_bounds__(256) awq_scale_activations_kernel(const __half* __restrict__ x,
                                                                const float* __restrict__ s, long long total8, int K,
                                                                __half* __restrict__ xs) {
-  pdl_enter();
+  pdl_enter_early();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= total8) return;
   const long long off = i * 8;

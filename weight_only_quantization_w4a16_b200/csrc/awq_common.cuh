@@ -62,6 +62,14 @@ __device__ __forceinline__ void pdl_enter() {
   pdl_wait();
   pdl_launch_dependents();
 }
+// The same for kernels that write nothing the next kernel may read before its own wait (it reads
+// this kernel's outputs only after griddepcontrol.wait, which returns once this grid has
+// completed): the next kernel launches at once, so a decode kernel after an activation kernel
+// can already stream its packed weights while the kernels before it run.
+__device__ __forceinline__ void pdl_enter_early() {
+  pdl_launch_dependents();
+  pdl_wait();
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
