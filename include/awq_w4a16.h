@@ -264,7 +264,11 @@ AWQ_API awq_status_t awq_search_alpha_noalloc(const uint16_t* x, const uint16_t*
 /* Synchronizes `stream`, then reads and clears the device status word of the
  * current device. Returns AWQ_ERR_TIMEOUT if a kernel since the last poll gave
  * up a bounded wait (its outputs are then undefined), AWQ_ERR_CUDA if the
- * stream reports an error, AWQ_OK otherwise. */
+ * stream reports an error, AWQ_OK otherwise.
+ * The status word is one per device, shared by every stream and launch of this
+ * library on it: a timeout raised by a kernel of another stream since the last
+ * poll is reported (and cleared) here too. With several streams, synchronize
+ * all of them before polling to attribute a timeout to the work just done. */
 AWQ_API awq_status_t awq_poll_device_status(awq_stream_t stream);
 
 /* Test hook: sets the time (ns) after which a bounded wait inside a kernel
