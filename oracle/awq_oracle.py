@@ -42,7 +42,11 @@ Readings where the pages are silent (each is also listed in the design notes):
   rint = round half to even, fp32 division;
 * dequantization ŵ = (q - z) * S, exact in float64; y = x' . ŵ^T in float64;
 * scale search: an even grid of 20 exponents over [0, 1); the squared Frobenius
-  error of the layer output on the calibration rows, against x . W^T, picks one.
+  error of the layer output on the calibration rows, against x . W^T, picks one;
+* variants ([AWQ-README] model-zoo table INT3-g128; [AutoAWQ-blog] w_bit,
+  q_group_size, zero_point): b-bit codes with qmax = 2^b - 1 in the same steps;
+  zero_point false (symmetric): S = fp16(max(max |w'|, 1e-5) / (2^(b-1) - 1)),
+  z = 2^(b-1) fixed, q = clamp(rint(w' / S) + z, 0, qmax); groups of 64 or 128.
 
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``
 (brute force, closed forms, invariants, exact rational arithmetic,
@@ -139,6 +143,60 @@ def quantize_groups(wf: np.ndarray) -> Tuple[np.ndarray, np.ndarray, np.ndarray]
     q = np.rint(w / Sf[..., None]) + z[..., None]
     q = np.fmin(np.fmax(q, np.float32(0)), np.float32(QMAX))
     return q.astype(np.uint8).reshape(N, K), S, z.astype(np.uint8)
+
+
+def quantize_groups_cfg(wf: np.ndarray, bits: int = BITS, group_size: int = GROUP_SIZE,
+                        zero_point: bool = True) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The quantizer for the configurations the pages name besides INT4-g128-asymmetric.
+
+    [AWQ-README] model-zoo table (INT3-g128 models next to INT4-g128),
+    [AutoAWQ-blog] "Quantizing a model with AutoAWQ" (``w_bit``, ``q_group_size``
+    = the group that shares one scale and one zero point, ``zero_point`` =
+    asymmetric quantization), [HF-AWQ] section 2 (bits, group_size, zero_point).
+
+    Returns q[N, K] (uint8, 0..2^bits - 1), S[N, K/group] (fp16), z[N, K/group]
+    (uint8). Per group, fp32 round to nearest even, with qmax = 2^bits - 1:
+
+    * zero_point true (asymmetric): the steps of ``quantize_groups`` with 15
+      replaced by qmax: S = fp16(max(hi - lo, 1e-5) / qmax),
+      z = clamp(rint(-lo / S), 0, qmax);
+    * zero_point false (symmetric): a = max(|lo|, |hi|),
+      S = fp16(max(a, 1e-5) / (2^(bits-1) - 1)), z = 2^(bits-1): the signed
+      code rint(w' / S) in [-2^(bits-1), 2^(bits-1) - 1] stored with the offset z;
+    * q = clamp(rint(w' / S) + z, 0, qmax) in both cases.
+    """
+    if bits not in (3, 4) or group_size not in (64, 128):
+        raise ValueError("bits must be 3 or 4 and group_size 64 or 128")
+    wf = np.asarray(wf, dtype=np.float16)
+    N, K = wf.shape
+    if K % group_size:
+        raise ValueError("K must be a multiple of the group size")
+    qmax = np.float32((1 << bits) - 1)
+    G = K // group_size
+    w = wf.astype(np.float32).reshape(N, G, group_size)
+    lo = np.fmin.reduce(w, axis=2)
+    hi = np.fmax.reduce(w, axis=2)
+    if zero_point:
+        S = (np.fmax(hi - lo, RANGE_FLOOR) / qmax).astype(np.float16)
+        Sf = S.astype(np.float32)
+        z = np.fmin(np.fmax(np.rint(-lo / Sf), np.float32(0)), qmax)
+    else:
+        a = np.fmax(np.abs(lo), np.abs(hi))
+        S = (np.fmax(a, RANGE_FLOOR) / np.float32((1 << (bits - 1)) - 1)).astype(np.float16)
+        Sf = S.astype(np.float32)
+        z = np.full(lo.shape, np.float32(1 << (bits - 1)))
+    q = np.rint(w / Sf[..., None]) + z[..., None]
+    q = np.fmin(np.fmax(q, np.float32(0)), qmax)
+    return q.astype(np.uint8).reshape(N, K), S, z.astype(np.uint8)
+
+
+def dequantize_cfg(q: np.ndarray, S: np.ndarray, z: np.ndarray, group_size: int) -> np.ndarray:
+    """ŵ = (q - z) * S with groups of ``group_size`` along K, exact in float64."""
+    N, K = q.shape
+    G = K // group_size
+    qg = q.astype(np.float64).reshape(N, G, group_size)
+    w = (qg - z.astype(np.float64)[..., None]) * S.astype(np.float64)[..., None]
+    return w.reshape(N, K)
 
 
 def dequantize(q: np.ndarray, S: np.ndarray, z: np.ndarray) -> np.ndarray:

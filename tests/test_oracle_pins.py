@@ -481,3 +481,94 @@ def test_split_qkv_blocks():
     y = np.arange(2 * 12).reshape(2, 12)
     q, k, v = O.split_qkv(y, 8, 2)
     assert q.tolist() == y[:, :8].tolist() and k.tolist() == y[:, 8:10].tolist() and v.tolist() == y[:, 10:].tolist()
+
+
+# ----------------------------------------------------------------------------
+# quantizer variants (INT3, symmetric, group 64)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("case", _load("quantizer_variant_cases.json")["groups"], ids=lambda c: c["name"])
+def test_quantizer_variant_hand_cases(case):
+    vals = list(case["values"]) + [case["fill"]] * (128 - len(case["values"]))
+    W = np.array([vals], dtype=np.float16)
+    assert np.all(W.astype(np.float64) == np.array([vals])), "fixture values must be fp16-exact"
+    q, S, z = O.quantize_groups_cfg(W, case["bits"], 128, case["zero_point"])
+    expect = list(case["codes"]) + [case["fill_code"]] * (128 - len(case["codes"]))
+    assert q[0].tolist() == expect
+    assert int(_f16_bits(S)[0, 0]) == int(case["scale_bits"], 16)
+    assert int(z[0, 0]) == case["zero"]
+
+
+def test_quantizer_cfg_default_is_the_pinned_int4_quantizer():
+    W = workloads.make_weight(0, 7, 1, 48, 512)
+    a = O.quantize_groups(W)
+    b = O.quantize_groups_cfg(W, 4, 128, True)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
+def _brute_codes_cfg(w32, S16, qmax, z_fixed=None):
+    """Nearest level c in 0..qmax of (c - z) to w/S, ties to the even integer; z as in _brute_codes
+    (nearest integer in 0..qmax to -lo/S) unless fixed."""
+    Sf = np.float32(S16)
+    if z_fixed is None:
+        t = float(np.float32(-np.float32(np.min(w32))) / Sf)
+        zb = min(range(qmax + 1), key=lambda c: (abs(t - c), c % 2))
+    else:
+        zb = z_fixed
+    out = []
+    for w in w32:
+        v = float(np.float32(w) / Sf)
+        out.append(min(range(qmax + 1), key=lambda c: (abs(v - (c - zb)), (c - zb) % 2)))
+    return np.array(out, dtype=np.uint8), zb
+
+
+@pytest.mark.parametrize("bits,zero_point", [(3, True), (3, False), (4, False)])
+def test_quantizer_variant_brute_force(bits, zero_point):
+    rng = np.random.default_rng(77 + bits + 10 * zero_point)
+    qmax = (1 << bits) - 1
+    for trial in range(40):
+        kind = trial % 4
+        if kind == 0:
+            w = rng.standard_normal(128) * 0.02
+        elif kind == 1:
+            w = rng.standard_normal(128) * 3.0 + rng.uniform(-2, 2)
+        elif kind == 2:
+            w = rng.uniform(0.5, 1.5, 128)
+        else:
+            w = -rng.uniform(0.5, 1.5, 128)
+        W = w.astype(np.float16)[None, :]
+        q, S, z = O.quantize_groups_cfg(W, bits, 128, zero_point)
+        w32 = W[0].astype(np.float32)
+        if not zero_point:
+            # the scale itself: fp16 of max|w| / (2^(bits-1) - 1)
+            a = float(np.max(np.abs(w32)))
+            assert S[0, 0] == np.float16(np.float32(a) / np.float32((1 << (bits - 1)) - 1))
+        qb, zb = _brute_codes_cfg(w32, S[0, 0], qmax, None if zero_point else 1 << (bits - 1))
+        assert int(z[0, 0]) == zb
+        assert np.array_equal(q[0], qb), f"trial {trial}"
+
+
+def test_quantizer_symmetric_invariants():
+    """Symmetric codes never clamp for finite groups: |w - (q - z) S| <= S/2 and q >= 1."""
+    W = workloads.make_weight(3, 7, 2, 64, 1024)
+    for bits in (3, 4):
+        q, S, z = O.quantize_groups_cfg(W, bits, 128, False)
+        assert np.all(z == (1 << (bits - 1)))
+        err = np.abs(O.dequantize_cfg(q, S, z, 128) - W.astype(np.float64))
+        half = np.repeat(S.astype(np.float64), 128, axis=1) / 2
+        assert np.all(err <= half * (1 + 1e-6))
+        assert q.min() >= 1 and q.max() <= (1 << bits) - 1
+
+
+def test_quantizer_group64_equals_group128_of_duplicated_halves():
+    """A 64-wide group's min, max and codes are those of a 128-wide group holding it twice."""
+    W = workloads.make_weight(5, 7, 3, 16, 512)
+    for bits, zp in ((4, True), (3, False)):
+        q64, S64, z64 = O.quantize_groups_cfg(W, bits, 64, zp)
+        halves = W.reshape(16, 8, 64)
+        dup = np.concatenate([halves, halves], axis=2).reshape(16, 1024)
+        q128, S128, z128 = O.quantize_groups_cfg(dup, bits, 128, zp)
+        assert np.array_equal(q64.reshape(16, 8, 64), q128.reshape(16, 8, 128)[:, :, :64])
+        assert np.array_equal(_f16_bits(S64), _f16_bits(S128)) and np.array_equal(z64, z128)
+        # and dequantization respects the group width
+        wh = O.dequantize_cfg(q64, S64, z64, 64)
+        assert np.array_equal(wh, O.dequantize_cfg(q128, S128, z128, 128).reshape(16, 8, 128)[:, :, :64].reshape(16, 512))
