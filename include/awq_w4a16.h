@@ -96,10 +96,12 @@ AWQ_API int awq_layout_version(void);
 /* Static, human-readable name of a status code. Never NULL. */
 AWQ_API const char* awq_status_string(int status);
 
-/* AWQ_OK iff (bits, group_size, zero_point) is the built configuration
- * (4, 128, 1) — the quantization_config of "transformers - AWQ" section 2 and
- * the quant_config of the AutoAWQ section of the llmstudio.ru page.
- * AWQ_ERR_UNSUPPORTED otherwise. Pure host function. */
+/* AWQ_OK iff (bits, group_size, zero_point) is a built configuration: bits 4
+ * or 3, group size 128, zero point 1 or 0 — (4, 128, 1) is the
+ * quantization_config of "transformers - AWQ" section 2 and the quant_config
+ * of the AutoAWQ section of the llmstudio.ru page; INT3-g128 is in the model
+ * zoo of the llm-awq README. AWQ_ERR_UNSUPPORTED otherwise (group size 64
+ * included). Pure host function. */
 AWQ_API awq_status_t awq_check_config(int bits, int group_size, int zero_point);
 
 /* Sizes in bytes of the packed arrays for an N x K layer: Ntiles*G2 times
@@ -144,6 +146,26 @@ AWQ_API awq_status_t awq_scale_activations(const uint16_t* x, const float* s, in
 AWQ_API awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K,
                                uint32_t* qweight, uint16_t* scales, uint8_t* zeros,
                                awq_stream_t stream);
+
+/* a2 variants: the same fold and group quantizer for the other configurations
+ * the pages name — INT3-g128 (model-zoo table of the llm-awq README) and the
+ * symmetric form (zero_point false; AutoAWQ section of the llmstudio.ru page:
+ * zero_point selects asymmetric quantization).
+ *   bits       4 or 3; 3-bit codes (0..7) occupy the same 4-bit slots of packed
+ *              layout v2 (same sizes, same linear kernels).
+ *   group_size 128 (64 returns AWQ_ERR_UNSUPPORTED: every kernel here works on
+ *              128-k groups; the oracle defines g64 for a future layout).
+ *   zero_point 1: asymmetric, S = fp16(max(hi - lo, 1e-5) / (2^bits - 1)),
+ *              z = clamp(rint(-lo / S), 0, 2^bits - 1);
+ *              0: symmetric, S = fp16(max(max|w'|, 1e-5) / (2^(bits-1) - 1)),
+ *              z = 2^(bits-1) (stored in `zeros` like any zero point);
+ *              q = clamp(rint(w' / S) + z, 0, 2^bits - 1) in both cases.
+ * Other arguments, layout, errors and the no-early-start rule as for
+ * awq_quantize_g128, which is awq_quantize(..., 4, 128, 1, ...). The linear
+ * entry points dequantize every variant as (q - z) * S unchanged. */
+AWQ_API awq_status_t awq_quantize(const uint16_t* W, const float* fold_scale, int N, int K, int bits,
+                                  int group_size, int zero_point, uint32_t* qweight, uint16_t* scales,
+                                  uint8_t* zeros, awq_stream_t stream);
 
 /* a3. Decode W4A16 linear layer (context: "Installation" step 3 of the llm-awq
  * README, W4A16 decode kernels).

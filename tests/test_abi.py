@@ -64,8 +64,18 @@ def test_check_config_against_page_configs(lib):
     assert lib.awq_check_config(hf["bits"], hf["group_size"], int(hf["zero_point"])) == 0
     aw = fx["autoawq_quant_config"]
     assert lib.awq_check_config(aw["w_bit"], aw["q_group_size"], int(aw["zero_point"])) == 0
+    for v in fx["supported_variants"]:
+        assert lib.awq_check_config(v["bits"], v["group_size"], int(v["zero_point"])) == 0
     for u in fx["unsupported_examples"]:
         assert lib.awq_check_config(u["bits"], u["group_size"], int(u["zero_point"])) == 2
+
+
+def test_quantize_variant_argument_checks(lib):
+    """awq_quantize rejects unbuilt configurations before any CUDA call (no GPU needed)."""
+    V = ctypes.c_void_p
+    for bits, group, zp in ((4, 64, 1), (8, 128, 1), (3, 64, 0)):
+        assert lib.awq_quantize(V(0x10000), None, 16, 256, bits, group, zp, V(0x10000), V(0x10000), V(0x10000), None) == 2
+    assert lib.awq_quantize(None, None, 16, 256, 3, 128, 0, V(0x10000), V(0x10000), V(0x10000), None) == 1
 
 
 @pytest.mark.parametrize("N,K", [(1, 128), (128, 128), (300, 256), (4096, 11008), (28672, 8192), (513, 640)])

@@ -62,6 +62,7 @@ _SIGS = {
     "awq_activation_scale": ([_VP, _I, _I, ctypes.c_float, _VP, _VP, _VP], _I),
     "awq_scale_activations": ([_VP, _VP, _I, _I, _VP, _VP], _I),
     "awq_quantize_g128": ([_VP, _VP, _I, _I, _VP, _VP, _VP, _VP], _I),
+    "awq_quantize": ([_VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP], _I),
     "awq_w4a16_gemv": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_w4a16_gemm": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
     "awq_w4a16_linear": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _VP], _I),
@@ -264,6 +265,21 @@ def awq_quantize_g128(W, fold_scale=None, out=None):
     st = load_library().awq_quantize_g128(_ptr(W), _ptr(fold_scale), N, K, _ptr(qweight), _ptr(scales),
                                           _ptr(zeros), _stream_ptr())
     _check("awq_quantize_g128", st)
+    return qweight, scales, zeros
+
+
+def awq_quantize(W, fold_scale=None, bits: int = 4, group_size: int = 128, zero_point: bool = True, out=None):
+    """a2 variants: INT4 or INT3 codes, asymmetric (zero_point) or symmetric, group size 128, in
+    packed layout v2. Returns (qweight, scales, zeros)."""
+    torch = _torch()
+    _need(W, torch.float16, "W", 2)
+    N, K = W.shape
+    out = out if out is not None else alloc_packed(N, K, W.device)
+    validate_quantize(W, fold_scale, out)
+    qweight, scales, zeros = out
+    st = load_library().awq_quantize(_ptr(W), _ptr(fold_scale), N, K, int(bits), int(group_size), int(bool(zero_point)),
+                                     _ptr(qweight), _ptr(scales), _ptr(zeros), _stream_ptr())
+    _check("awq_quantize", st)
     return qweight, scales, zeros
 
 

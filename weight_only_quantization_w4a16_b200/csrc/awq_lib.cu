@@ -540,7 +540,9 @@ const char* awq_status_string(int status) {
 }
 
 awq_status_t awq_check_config(int bits, int group_size, int zero_point) {
-  return (bits == 4 && group_size == kGroup && zero_point == 1) ? AWQ_OK : AWQ_ERR_UNSUPPORTED;
+  return ((bits == 4 || bits == 3) && group_size == kGroup && (zero_point == 0 || zero_point == 1))
+             ? AWQ_OK
+             : AWQ_ERR_UNSUPPORTED;
 }
 
 size_t awq_qweight_bytes(int N, int K) {
@@ -594,10 +596,11 @@ awq_status_t awq_scale_activations(const uint16_t* x, const float* s, int M, int
                    reinterpret_cast<__half*>(x_scaled));
 }
 
-awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K, uint32_t* qweight,
-                               uint16_t* scales, uint8_t* zeros, awq_stream_t stream) {
+awq_status_t awq_quantize(const uint16_t* W, const float* fold_scale, int N, int K, int bits, int group_size,
+                          int zero_point, uint32_t* qweight, uint16_t* scales, uint8_t* zeros, awq_stream_t stream) {
   if (!W || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
   if (K < kGroup || K % kGroup != 0 || !rows_ok(N, K)) return AWQ_ERR_INVALID_ARG;
+  if (awq_check_config(bits, group_size, zero_point) != AWQ_OK) return AWQ_ERR_UNSUPPORTED;
   if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(fold_scale))
     return AWQ_ERR_MISALIGNED;
   int dev, sms;
@@ -617,20 +620,29 @@ awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return AWQ_ERR_CUDA;
   }
-  static std::atomic<uint64_t> done_f{0}, done_n{0};
-  st = fold_scale ? ensure_smem(awq_quantize_g128_kernel<true>, kQSmem, dev, done_f)
-                  : ensure_smem(awq_quantize_g128_kernel<false>, kQSmem, dev, done_n);
-  if (st != AWQ_OK) return st;
   const long long units = static_cast<long long>(padded_rows(N) / kSuperRows) * (K / kGroup);
   const int grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(AWQ_QUANT_MINBLOCKS) * sms));
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (fold_scale)
-    return launch_ex(awq_quantize_g128_kernel<true>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), dim3(0, 0, 0), kQSmem, s,
-                     map,
-                     fold_scale, N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
-  return launch_ex(awq_quantize_g128_kernel<false>, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), dim3(0, 0, 0), kQSmem, s,
-                   map,
-                   static_cast<const float*>(nullptr), N, K, qweight, reinterpret_cast<__half*>(scales), zeros);
+  auto run = [&](auto kernel, std::atomic<uint64_t>& done) -> awq_status_t {
+    const awq_status_t e = ensure_smem(kernel, kQSmem, dev, done);
+    if (e != AWQ_OK) return e;
+    return launch_ex(kernel, dim3(grid, 1, 1), dim3(kQThreads, 1, 1), dim3(0, 0, 0), kQSmem, s, map, fold_scale, N, K,
+                     qweight, reinterpret_cast<__half*>(scales), zeros);
+  };
+  static std::atomic<uint64_t> done[8];
+  const bool f = fold_scale != nullptr;
+  const int variant = (bits == 3 ? 2 : 0) + (zero_point ? 0 : 1);
+  switch (variant) {
+    case 0: return f ? run(awq_quantize_g128_kernel<true, 4, false>, done[0]) : run(awq_quantize_g128_kernel<false, 4, false>, done[1]);
+    case 1: return f ? run(awq_quantize_g128_kernel<true, 4, true>, done[2]) : run(awq_quantize_g128_kernel<false, 4, true>, done[3]);
+    case 2: return f ? run(awq_quantize_g128_kernel<true, 3, false>, done[4]) : run(awq_quantize_g128_kernel<false, 3, false>, done[5]);
+    default: return f ? run(awq_quantize_g128_kernel<true, 3, true>, done[6]) : run(awq_quantize_g128_kernel<false, 3, true>, done[7]);
+  }
+}
+
+awq_status_t awq_quantize_g128(const uint16_t* W, const float* fold_scale, int N, int K, uint32_t* qweight,
+                               uint16_t* scales, uint8_t* zeros, awq_stream_t stream) {
+  return awq_quantize(W, fold_scale, N, K, 4, kGroup, 1, qweight, scales, zeros, stream);
 }
 
 awq_status_t awq_w4a16_gemv(const uint16_t* x, const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros,

@@ -10,6 +10,11 @@
 //   S   = fp16(max(hi - lo, 1e-5) / 15)
 //   z   = clamp(rint(-lo / S), 0, 15)
 //   q   = clamp(rint(w' / S) + z, 0, 15)
+// Variants (template arguments kBits, kSym; the llm-awq README's model zoo lists INT3-g128
+// next to INT4-g128, the llmstudio.ru AutoAWQ section names w_bit and zero_point): 3-bit codes
+// take qmax = 7 in place of 15 in the same rules (stored in the same 4-bit slots); the symmetric
+// form (zero_point false) takes S = fp16(max(max|w'|, 1e-5) / (2^(b-1) - 1)) and the fixed
+// z = 2^(b-1), then the same q = clamp(rint(w' / S) + z, 0, qmax).
 //
 // w'/S is computed as va = w'*r, rho = fma(-S, va, w'), v = fma(rho, r, va)
 // with r = RN(1/S), on packed fp32 pairs. This equals the IEEE quotient RN(w'/S) for every fp16
@@ -106,7 +111,9 @@ constexpr int kQComputeWarps = 8;
 constexpr int kQThreads = (kQComputeWarps + 1) * 32;        // + 1 producer warp
 constexpr int kQSmem = kQStages * kQStageBytes + 2 * kQStages * 8 + 16 + 1024;
 
-template <bool kFold>
+// kBits: 4 or 3 (codes 0..2^kBits - 1 in the same 4-bit slots); kSym: symmetric variant
+// (S = fp16(max(max|w'|, 1e-5) / (2^(kBits-1) - 1)), z = 2^(kBits-1)), the asymmetric rules otherwise.
+template <bool kFold, int kBits = 4, bool kSym = false>
 __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g128_kernel(const __grid_constant__ CUtensorMap tmap_w,
                                                                  const float* __restrict__ fold, int N, int K,
                                                                  uint32_t* __restrict__ qweight,
@@ -238,13 +245,23 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
     hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, 8));
 
     // ---- scale, zero point, reciprocal
-    const float range = fmaxf(__fsub_rn(hi, lo), 1e-5f);
-    const __half S = __float2half_rn(__fdiv_rn(range, 15.0f));
+    constexpr int kQMax = (1 << kBits) - 1;
+    constexpr float kQMaxF = static_cast<float>(kQMax);
+    __half S;
+    float zf;
+    if constexpr (kSym) {
+      const float amax = fmaxf(fmaxf(fabsf(lo), fabsf(hi)), 1e-5f);
+      S = __float2half_rn(__fdiv_rn(amax, static_cast<float>((1 << (kBits - 1)) - 1)));
+      zf = static_cast<float>(1 << (kBits - 1));
+    } else {
+      const float range = fmaxf(__fsub_rn(hi, lo), 1e-5f);
+      S = __float2half_rn(__fdiv_rn(range, kQMaxF));
+      zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, __half2float(S))), 0.0f), kQMaxF);
+    }
     const float Sf = __half2float(S);
-    const float zf = fminf(fmaxf(rintf(__fdiv_rn(-lo, Sf)), 0.0f), 15.0f);
     const float rcp = __frcp_rn(Sf);
-    // clamp(rint(v) + z, 0, 15) == rint(clamp(v, -z, 15 - z)) + z, as -z and 15 - z are integers
-    const float vlo = -zf, vhi = __fsub_rn(15.0f, zf);
+    // clamp(rint(v) + z, 0, qmax) == rint(clamp(v, -z, qmax - z)) + z, as -z and qmax - z are integers
+    const float vlo = -zf, vhi = __fsub_rn(kQMaxF, zf);
     const uint64_t rcp2 = f2_pack(rcp, rcp), nS2 = f2_pack(-Sf, -Sf), magic2 = f2_pack(kRoundMagic, kRoundMagic);
     const uint32_t zsub = (16u - static_cast<uint32_t>(__float2int_rz(zf))) * 0x01010101u;
 
@@ -272,9 +289,11 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
             const uint64_t v2 = f2_fma(rho, rcp2, va);
             const float2 tq = f2_unpack(f2_add(v2, magic2));
             const uint32_t t16 = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x5410);
-            code2[pr] = __viaddmin_s16x2_relu(t16, zoff2, 0x000F000Fu);   // max(min(n + z, 15), 0)
+            code2[pr] = __viaddmin_s16x2_relu(t16, zoff2, kQMax * 0x00010001u);   // max(min(n + z, qmax), 0)
           }
-          quad[i][sbh] = __byte_perm(code2[0], code2[1], 0x6420);
+          // padding rows (n >= N) read as zeros: code 0 unless the zero point is fixed (symmetric)
+          if constexpr (kSym) quad[i][sbh] = valid ? __byte_perm(code2[0], code2[1], 0x6420) : 0u;
+          else quad[i][sbh] = __byte_perm(code2[0], code2[1], 0x6420);
         }
       }
     } else {
@@ -291,12 +310,18 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
             const uint64_t va = f2_mul(w2, rcp2);
             const uint64_t rho = f2_fma(nS2, va, w2);
             float2 v = f2_unpack(f2_fma(rho, rcp2, va));
+            if constexpr (kSym) {
+              // S = inf (an overflowed fold) gives rcp = 0: the IEEE quotient is w * 0 (0 for finite w,
+              // NaN for infinite w), while the correction term above is NaN; with the fixed zero point
+              // the two give different codes, so take the quotient itself
+              if (rcp == 0.0f) v = f2_unpack(va);
+            }
             v.x = fminf(fmaxf(v.x, vlo), vhi);
             v.y = fminf(fmaxf(v.y, vlo), vhi);
             const float2 tq = f2_unpack(f2_add(f2_pack(v.x, v.y), magic2));
             lowbytes[pr] = __byte_perm(__float_as_uint(tq.x), __float_as_uint(tq.y), 0x0040);
           }
-          // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, 15], no borrows
+          // bytes (16 + n) for slots e0..e3, minus (16 - z) per byte: n + z in [0, qmax], no borrows
           const uint32_t q4 = __byte_perm(lowbytes[0], lowbytes[1], 0x5410) - zsub;
           quad[i][sbh] = valid ? q4 : 0u;
         }
