@@ -87,7 +87,9 @@ typedef enum {
   AWQ_ERR_UNSUPPORTED = 2,   /* configuration or device not built (bits != 4, group != 128, ...) */
   AWQ_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
   AWQ_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
-  AWQ_ERR_TIMEOUT = 5        /* a kernel gave up a bounded wait (reported by awq_poll_device_status) */
+  AWQ_ERR_TIMEOUT = 5,       /* a kernel gave up a bounded wait (reported by awq_poll_device_status) */
+  AWQ_ERR_BOUNDS = 6         /* debug builds (-DAWQ_DEBUG_BOUNDS) only: a kernel's index check failed and
+                                the access was skipped (reported by awq_poll_device_status) */
 } awq_status_t;
 
 /* Packed-layout version; bumps whenever the layout above changes. */
@@ -286,7 +288,8 @@ AWQ_API awq_status_t awq_search_alpha_noalloc(const uint16_t* x, const uint16_t*
 /* Synchronizes `stream`, then reads and clears the device status word of the
  * current device. Returns AWQ_ERR_TIMEOUT if a kernel since the last poll gave
  * up a bounded wait (its outputs are then undefined), AWQ_ERR_CUDA if the
- * stream reports an error, AWQ_OK otherwise.
+ * stream reports an error, AWQ_ERR_BOUNDS (debug builds only) if a kernel's
+ * index check failed, AWQ_OK otherwise.
  * The status word is one per device, shared by every stream and launch of this
  * library on it: a timeout raised by a kernel of another stream since the last
  * poll is reported (and cleared) here too. With several streams, synchronize

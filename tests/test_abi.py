@@ -50,9 +50,20 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name)
 
 
+def test_debug_bounds_library_exports_the_same_symbols():
+    """The -DAWQ_DEBUG_BOUNDS build (built by build(); the GPU tests run it) has the same ABI."""
+    from weight_only_quantization_w4a16_b200 import build as B
+    path = B.build(debug_bounds=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (awq_\w+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+    dbg = ctypes.CDLL(path)
+    assert dbg.awq_layout_version() == 2
+
+
 def test_layout_version_and_status_strings(lib):
     assert lib.awq_layout_version() == 2
-    for code in range(6):
+    for code in range(7):
         s = lib.awq_status_string(code).decode()
         assert s.startswith("AWQ_")
     assert lib.awq_status_string(99).decode() == "AWQ_ERR_UNKNOWN"

@@ -35,6 +35,7 @@ AWQ_ERR_UNSUPPORTED = 2
 AWQ_ERR_MISALIGNED = 3
 AWQ_ERR_CUDA = 4
 AWQ_ERR_TIMEOUT = 5
+AWQ_ERR_BOUNDS = 6    # debug builds only
 
 GROUP_SIZE = 128
 BITS = 4

@@ -15,6 +15,9 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libawq_w4a16.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+# the same library with the kernels' index checks compiled in (-DAWQ_DEBUG_BOUNDS): a failed check
+# is reported by awq_poll_device_status as AWQ_ERR_BOUNDS instead of touching memory out of bounds
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libawq_w4a16_debug_bounds.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -35,10 +38,10 @@ def _sources():
     return out
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB_PATH):
+def needs_build(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
@@ -49,10 +52,14 @@ def nvcc_path() -> str:
     return cand
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and not needs_build():
-        return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug_bounds: bool = False) -> str:
+    """Compiles the library (or its bounds-checking debug variant) if a source is newer."""
+    out = DEBUG_LIB_PATH if debug_bounds else LIB_PATH
+    if debug_bounds:
+        extra_flags = (*extra_flags, "-DAWQ_DEBUG_BOUNDS")
+    if not force and not needs_build(out):
+        return out
+    tmp = out + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, *extra_flags,
            "-I", INCLUDE, "-I", CSRC,
            "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map"),
@@ -64,10 +71,11 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr, flush=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
-          extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+          extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [],
+          debug_bounds="--debug-bounds" in sys.argv)

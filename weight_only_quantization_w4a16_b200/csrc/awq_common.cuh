@@ -36,6 +36,7 @@ __host__ __device__ inline int padded_rows(int N) { return ceil_div(N, kSuperRow
 // Device status word and the wait budget for bounded spin-waits.
 // ---------------------------------------------------------------------------
 constexpr int kDevStatusTimeout = 1;
+constexpr int kDevStatusBounds = 2;   // debug builds: a kernel's bounds check failed
 constexpr unsigned long long kDefaultWaitBudgetNs = 2000000000ull;   // 2 s
 constexpr unsigned long long kDrainBudgetNs = 1000000000ull;         // 1 s for teardown waits
 
@@ -45,6 +46,19 @@ __device__ unsigned long long g_wait_budget_ns = kDefaultWaitBudgetNs;
 // Test hook: nonzero makes the producer of each pipelined kernel skip the copies of its first
 // ring stage, so the consumers' wait on that stage can only end by running out its budget.
 __device__ int g_debug_drop_first_copy = 0;
+
+// Debug builds (-DAWQ_DEBUG_BOUNDS) check the kernels' computed offsets against the extents of the
+// buffers they address: a failed check records kDevStatusBounds in the device status word and the
+// access is skipped (no trap, no fault). In normal builds AWQ_CHECK(cond) is the constant true.
+#ifdef AWQ_DEBUG_BOUNDS
+__device__ __forceinline__ bool awq_check(bool ok) {
+  if (!ok) atomicOr(&g_dev_status, kDevStatusBounds);
+  return ok;
+}
+#define AWQ_CHECK(cond) ::awq::awq_check(cond)
+#else
+#define AWQ_CHECK(cond) true
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -220,6 +220,10 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, MINB)
     if (lane == 0) {
       auto issue_weights = [&](int slot, const Cursor& c) {
         const int np = stage_np(c);
+        // the stage's (tile, pair) range lies inside the packed arrays and the ring slot
+        if (!AWQ_CHECK(tile_of(c.u) >= 0 && tile_of(c.u) < a.units && c.p >= 0 && np >= 1 && c.p + np <= G2 &&
+                       np <= SB && slot >= 0 && slot < S))
+          return;
         uint8_t* sb = smem + static_cast<size_t>(slot) * a.stage_bytes;
         mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(np * (2048 + 64 + 16) + a.x_box_bytes));
         const size_t tp = static_cast<size_t>(tile_of(c.u)) * G2 + c.p;   // (tile, pair) index
@@ -275,6 +279,7 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, MINB)
     float* rec = rec_all + static_cast<size_t>(warp) * R * rec_elems;
     int ri = 0;
     auto flush = [&]() {
+      if (!AWQ_CHECK(ri >= 0 && ri < R)) return;
       float* pr = rec + ri * rec_elems;
 #pragma unroll
       for (int j = 0; j < MT; ++j)
@@ -340,6 +345,7 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, MINB)
   // element e of relative unit ur summed over this CTA's warps (zero for a unit it did not touch)
   auto cta_sum = [&](int ur, int e) -> float {
     if (ur < uf || ur > ul) return 0.f;
+    if (!AWQ_CHECK(ur - uf < R && e >= 0 && e < rec_elems)) return 0.f;
     const float* pr = rec_all + static_cast<size_t>(ur - uf) * rec_elems + e;
     float v = 0.f;
 #pragma unroll 4
@@ -368,7 +374,7 @@ __global__ void __launch_bounds__(GemvCfg<CW, SBW, kSwz>::kThreads, MINB)
     else {
       if (live && shared_blk) {
         float* dst = cluster.map_shared_rank(recv, 0);
-        for (int idx = threadIdx.x; idx < upc * rec_elems; idx += blockDim.x)
+        for (int idx = threadIdx.x; idx < upc * rec_elems && AWQ_CHECK(idx < 2 * rec_elems); idx += blockDim.x)
           dst[idx] = cta_sum(bb * upc + idx / rec_elems, idx % rec_elems);
       }
       cluster_arrive();                                      // release: the pushed sums

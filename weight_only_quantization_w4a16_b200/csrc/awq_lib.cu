@@ -535,6 +535,7 @@ const char* awq_status_string(int status) {
     case AWQ_ERR_MISALIGNED: return "AWQ_ERR_MISALIGNED: pointer not 16-byte aligned";
     case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA runtime error";
     case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case AWQ_ERR_BOUNDS: return "AWQ_ERR_BOUNDS: a bounds check of the debug build failed";
     default: return "AWQ_ERR_UNKNOWN";
   }
 }
@@ -800,7 +801,8 @@ awq_status_t awq_poll_device_status(awq_stream_t stream) {
   if (v == 0) return AWQ_OK;
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int)) != cudaSuccess) return AWQ_ERR_CUDA;
-  return (v & kDevStatusTimeout) ? AWQ_ERR_TIMEOUT : AWQ_ERR_CUDA;
+  if (v & kDevStatusTimeout) return AWQ_ERR_TIMEOUT;
+  return (v & kDevStatusBounds) ? AWQ_ERR_BOUNDS : AWQ_ERR_CUDA;
 }
 
 awq_status_t awq_debug_drop_first_copy(int enable) {

@@ -332,7 +332,8 @@ __global__ void __launch_bounds__(kQThreads, AWQ_QUANT_MINBLOCKS) awq_quantize_g
     // Chunk i covers k-tile (i >> 2), column block t = (i & 3), steps s = 2*half + sbh.
     // Tile T = 8 st + nt of packed layout v2: its k-tiles follow one another (KTp per tile).
     const int T = st * 8 + nt;
-    if (T < ntiles) {
+    // the group's codes lie inside the packed arrays (ntiles x KTp chunks of 512 bytes)
+    if (T < ntiles && AWQ_CHECK(g >= 0 && g < G && 2 * g + h < KTp)) {
       uint32_t* out = qweight + (static_cast<size_t>(T) * KTp + 2 * g + h) * kChunkWords;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
