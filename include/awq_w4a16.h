@@ -310,6 +310,15 @@ AWQ_API awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns);
  * 0 restores normal operation. Synchronous; current device. */
 AWQ_API awq_status_t awq_debug_drop_first_copy(int enable);
 
+/* Test hook: the prefill kernel's K split. 0 (the default) lets the
+ * library's round model choose, per launch, whether the two CTAs of a
+ * thread-block cluster share each output tile (each over half of K, their
+ * fp32 partial sums added in a fixed order); 1 never splits, 2 always
+ * splits. Results agree within fp32 rounding of the split sum. Host-side
+ * setting for all devices, read at each launch; AWQ_ERR_INVALID_ARG for
+ * other values. */
+AWQ_API awq_status_t awq_debug_set_gemm_split(int ks);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -81,6 +81,14 @@ def test_check_config_against_page_configs(lib):
         assert lib.awq_check_config(u["bits"], u["group_size"], int(u["zero_point"])) == 2
 
 
+def test_gemm_split_hook_is_host_only(lib):
+    """The K-split test hook takes 0, 1 or 2 and touches no device."""
+    for bad in (-1, 3, 100):
+        assert lib.awq_debug_set_gemm_split(bad) == 1
+    for ok in (2, 1, 0):
+        assert lib.awq_debug_set_gemm_split(ok) == 0
+
+
 def test_quantize_variant_argument_checks(lib):
     """awq_quantize rejects unbuilt configurations before any CUDA call (no GPU needed)."""
     V = ctypes.c_void_p

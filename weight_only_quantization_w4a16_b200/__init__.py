@@ -18,7 +18,7 @@ Functions (same names as the C ABI):
 * ``awq_w4a16_linear_silu_mul(x, qweight, scales, zeros, I)`` -> h = SiLU(gate) * up
 * ``awq_search_alpha(x, W, alphas)`` -> (err[n] float64, best index): the AWQ scale search
 * ``awq_poll_device_status()``, test hooks ``awq_debug_set_wait_budget_ns(ns)``,
-  ``awq_debug_drop_first_copy(enable)``
+  ``awq_debug_drop_first_copy(enable)``, ``awq_debug_set_gemm_split(ks)``
 """
 from __future__ import annotations
 
@@ -75,6 +75,7 @@ _SIGS = {
     "awq_search_alpha_noalloc": ([_VP, _VP, _I, _I, _I, _VP, _I, _VP, _VP, _VP], _I),
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
     "awq_debug_drop_first_copy": ([_I], _I),
+    "awq_debug_set_gemm_split": ([_I], _I),
 }
 
 
@@ -426,6 +427,11 @@ def awq_debug_set_wait_budget_ns(ns: int) -> None:
 
 def awq_debug_drop_first_copy(enable: bool) -> None:
     _check("awq_debug_drop_first_copy", load_library().awq_debug_drop_first_copy(int(bool(enable))))
+
+
+def awq_debug_set_gemm_split(ks: int) -> None:
+    """Prefill K split: 0 chooses per launch, 1 never splits, 2 always splits (a CTA pair per tile)."""
+    _check("awq_debug_set_gemm_split", load_library().awq_debug_set_gemm_split(int(ks)))
 
 
 class AWQLinear:

@@ -129,6 +129,30 @@ __device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity
       : "memory");
   return ok != 0;
 }
+// The same two waits with acquire semantics at cluster scope: for phases completed by arrivals
+// of the other CTA of a cluster, whose shared-memory stores into this CTA they make visible.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_for_cluster(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
 
 // Budgets below this (set only through the test hook) also bound each suspended try_wait, so
 // that the budget is honoured even when the hardware's own suspend window is longer.
@@ -137,11 +161,17 @@ constexpr unsigned long long kShortBudgetNs = 1000000ull;
 // Bounded wait: returns true when the phase with `parity` has completed.
 // Gives up (returns false) when *abort is set by another warp, or after
 // `budget_ns` of waiting, in which case it sets *abort and the device status.
+// kCluster: acquire at cluster scope (arrivals from the other CTA of a cluster).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   unsigned long long budget_ns) {
   const bool short_budget = budget_ns < kShortBudgetNs;
   const uint32_t hint = static_cast<uint32_t>(budget_ns);
-  auto try_once = [&]() { return short_budget ? mbar_try_wait_for(bar, parity, hint) : mbar_try_wait(bar, parity); };
+  auto try_once = [&]() {
+    if (kCluster)
+      return short_budget ? mbar_try_wait_for_cluster(bar, parity, hint) : mbar_try_wait_cluster(bar, parity);
+    return short_budget ? mbar_try_wait_for(bar, parity, hint) : mbar_try_wait(bar, parity);
+  };
   if (try_once()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -153,6 +183,39 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
       return false;
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: the cluster barrier, split into arrive and wait (all 32 lanes of a warp
+// execute each together), and shared-memory access to the other CTAs of the cluster.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of this CTA's shared-memory object `p` in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t cluster_smem_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// One arrival, with release semantics at cluster scope, on an mbarrier of another CTA.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// An asynchronous 16-byte store into another CTA's shared memory that completes 16 bytes of the
+// transaction count of `cluster_bar`, an mbarrier in that same CTA.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------

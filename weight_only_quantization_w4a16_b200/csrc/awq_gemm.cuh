@@ -72,11 +72,15 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 // CPS: resident CTAs per SM. With 2, each CTA keeps one TMEM accumulator (the other CTA's
 // epilogue and mainloop interleave with its own); with 1, two accumulators let the epilogue of
 // one tile overlap the mainloop of the next.
-template <int BT, int STAGES, int NDQ, int CPS = 1>
+// KS: CTAs that share one output tile, each over its part of K (a cluster of KS = 2 CTAs; rank 1
+// pushes its fp32 partial sums into rank 0's shared memory with asynchronous stores that count
+// down rank 0's mbarrier, 32 columns at a time, through an exchange buffer of two or more slots).
+template <int BT, int STAGES, int NDQ, int CPS = 1, int KS = 1>
 struct GemmCfg {
   static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
   static_assert(CPS == 1 || CPS == 2, "CTAs per SM");
   static_assert(NDQ == 4 || NDQ == 8, "dequant warps");
+  static_assert(KS == 1 || (KS == 2 && CPS == 1), "K split across a CTA pair");
   static constexpr int kA = kSuperRows * kKTile * 2;        // 16 KB dequantized weights
   static constexpr int kB = BT * kKTile * 2;                // x' tile
   static constexpr int kRawQ = kSuperChunkWords * 4;        // 4096 B
@@ -89,9 +93,16 @@ struct GemmCfg {
   static constexpr int kOffQ = kOffB + STAGES * kB;
   static constexpr int kOffS = kOffQ + STAGES * kRawQ;
   static constexpr int kOffZ = kOffS + STAGES * kRawS;
-  static constexpr int kOffBar = (kOffZ + STAGES * kRawZ + 15) / 16 * 16;
-  // barriers: full[S], aready[S], empty[S], accfull[2], accempty[2], drain[1]
-  static constexpr int kNumBars = 3 * STAGES + 5;
+  static constexpr int kXChunk = kSuperRows * 32 * 4;          // 16 KB: 32 fp32 columns of 128 rows
+  static constexpr int kOffX = (kOffZ + STAGES * kRawZ + 127) / 128 * 128;   // KS = 2: exchange slots
+  // KS = 2: as many exchange slots (up to one per 32-column chunk of the tile) as shared memory
+  // holds beside the ring
+  static constexpr int kXFree = (232448 - 1024 - 512 - kOffX) / kXChunk;
+  static constexpr int kXSlots = KS != 2 ? 0 : (BT / 32 < kXFree ? BT / 32 : kXFree);
+  static_assert(KS != 2 || kXSlots >= 1, "exchange slots");
+  static constexpr int kOffBar = kOffX + kXSlots * kXChunk;
+  // barriers: full[S], aready[S], empty[S], accfull[2], accempty[2], drain[1]; KS = 2: xfull[X], xempty[X]
+  static constexpr int kNumBars = 3 * STAGES + 5 + 2 * kXSlots;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16 + 1024;        // + slack for 1024-byte alignment
   // two accumulators of BT columns; tcgen05.alloc takes a power of two >= 32 columns
@@ -108,12 +119,12 @@ struct GemmCfg {
   static_assert(CPS == 1 || (kSmem + 1024) * 2 <= 233472, "two CTAs per SM must fit in shared memory");
 };
 
-template <int BT, int STAGES, int NDQ, int CPS, int EPI>
-__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
+template <int BT, int STAGES, int NDQ, int CPS, int EPI, int KS = 1>
+__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS>::kThreads, CPS)
     awq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
                     const EpiArgs epi, int M, int N, int K) {
-  using C = GemmCfg<BT, STAGES, NDQ, CPS>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -123,6 +134,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   uint64_t* accfull = bars + 3 * STAGES;
   uint64_t* accempty = accfull + 2;
   uint64_t* drain = accfull + 4;
+  uint64_t* xfull = drain + 1;                 // KS = 2, rank 0: rank 1's partial sums are in slot b
+  uint64_t* xempty = drain + 1 + C::kXSlots;   // KS = 2, rank 1: rank 0 has read slot b
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -134,6 +147,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   const int MTT = (M + BT - 1) / BT;
   const int ntiles = NST * MTT;
   const int KB = K / kKTile;
+  // KS = 2: the CTA pair of a cluster takes the same tiles, rank r the 64-k steps [kb0, kb1)
+  const int rank = KS == 2 ? static_cast<int>(blockIdx.x % KS) : 0;
+  const int tile0 = static_cast<int>(blockIdx.x) / KS, tstep = static_cast<int>(gridDim.x) / KS;
+  const int kb0 = rank * KB / KS, kb1 = (rank + 1) * KB / KS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -146,6 +163,11 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
       mbar_init(&accempty[b], 4);
     }
     mbar_init(drain, 1);
+    if (KS == 2)
+      for (int b = 0; b < C::kXSlots; ++b) {
+        mbar_init(&xfull[b], 1);    // rank 0's expect_tx arrival + 16 KB of rank 1's stores
+        mbar_init(&xempty[b], 4);   // one arrival per epilogue warp of rank 0
+      }
     *s_abort = 0;
     mbar_fence_init();
   }
@@ -162,6 +184,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (KS == 2) {   // the partner's barriers are initialised before any arrival on them
+    cluster_arrive();
+    cluster_wait();
+  }
   pdl_enter();
   const uint32_t tmem_base = *s_tmem;
   const unsigned long long budget = g_wait_budget_ns;
@@ -173,9 +199,9 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_par = 0;   // per stage: loaded at least once / parity of last load
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
         const int st = tile % NST, mt = tile / NST;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::kTx);
           if (EPI == kEpiSiluMul) {   // 4-tile boxes: gate tiles to slots 0..3, up tiles to slots 4..7
@@ -212,13 +238,13 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
       uint32_t phase = 0;
       bool ok = true, any = false;
       int it = 0;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
         const int b = it % C::kNAcc;
         const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
         if (!mbar_wait_bounded(&accempty[b], (use & 1) ^ 1, s_abort, budget)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BT);
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget) ||
               !mbar_wait_bounded(&aready[stage], phase, s_abort, budget)) { ok = false; break; }
           tc_fence_after();
@@ -227,7 +253,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
 #pragma unroll
           for (int kk = 0; kk < kKTile / 16; ++kk)
             tc_mma_f16(d_tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), idesc,
-                       (kb | kk) != 0 ? 1u : 0u);
+                       (kb != kb0 || kk != 0) ? 1u : 0u);
           any = true;
           tc_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -246,8 +272,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-      for (int kb = 0; kb < KB; ++kb) {
+    for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         // warp-uniform result: the code below needs the whole warp
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, s_abort, budget))) { ok = false; break; }
         const uint32_t* rq = reinterpret_cast<const uint32_t*>(smem + C::kOffQ + stage * C::kRawQ);
@@ -295,7 +321,8 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
     const int e = warp - C::kWarpEpi0;   // == warp % 4: TMEM lane quarter of this warp
     bool ok = true;
     int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+    uint32_t xq = 0;   // KS = 2: exchange chunks so far (slot xq % X, phase parity (xq / X) & 1)
+    for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
       const int st = tile % NST, mt = tile / NST;
       const int b = it % C::kNAcc;
       const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
@@ -310,6 +337,42 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * e) << 16) + static_cast<uint32_t>(b * BT + 32 * cc), v);
         tc_wait_ld();
+        if constexpr (KS == 2) {
+          // row 32 e + lane of the chunk: 8 16-byte pieces, piece j at position j ^ (lane & 7) of
+          // the row's 128 bytes (the 8 lanes of a shared-memory phase hit distinct banks)
+          const int xs = static_cast<int>(xq % C::kXSlots);
+          const uint32_t xpar = (xq / C::kXSlots) & 1;
+          ++xq;
+          uint8_t* xrow = smem + C::kOffX + xs * C::kXChunk + (32 * e + lane) * 128;
+          if (rank == 1) {
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<true>(&xempty[xs], xpar ^ 1, s_abort, budget))) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = cluster_smem_addr(xrow, 0);
+            const uint32_t bar = cluster_smem_addr(&xfull[xs], 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              st_async_v4(dst + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3], bar);
+            continue;   // rank 0 stores the tile
+          }
+          // one thread announces the chunk's bytes (rank 1's stores may count down before this)
+          if (e == 0 && lane == 0) mbar_arrive_expect_tx(&xfull[xs], C::kXChunk);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded<true>(&xfull[xs], xpar, s_abort, budget))) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {   // own partial sums first, then rank 1's (a fixed order)
+            const float4 p = *reinterpret_cast<const float4*>(xrow + ((j ^ (lane & 7)) << 4));
+            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + p.x);
+            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + p.y);
+            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + p.z);
+            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + p.w);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(cluster_smem_addr(&xempty[xs], 1));
+        }
         const int mb = mt * BT + 32 * cc;
         if (EPI == kEpiSiluMul) {
           const int I = N / 2;
@@ -339,6 +402,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS>::kThreads, CPS)
   if (warp == C::kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if (KS == 2) {   // neither CTA exits while the other may still write to or arrive on it
+    cluster_arrive();
+    cluster_wait();
   }
 }
 

@@ -43,18 +43,6 @@
 
 namespace awq {
 
-// ------------------------------------------------------------------------------------
-// Cluster barrier, split into arrive and wait (all 32 lanes of a warp execute each together).
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 // Per-launch arguments of the decode kernel.
 struct GemvArgs {
   const uint8_t* qweight;   // packed codes (layout v2), 2048 bytes per (tile, group pair)

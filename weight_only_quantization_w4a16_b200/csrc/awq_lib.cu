@@ -372,11 +372,11 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
-template <int BT, int STAGES, int NDQ, int CPS = 1, int EPI = kEpiPlain>
+template <int BT, int STAGES, int NDQ, int CPS = 1, int EPI = kEpiPlain, int KS = 1>
 awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using C = GemmCfg<BT, STAGES, NDQ, CPS>;
-  auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS, EPI>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS>;
+  auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS, EPI, KS>;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, C::kSmem, dev, smem_done);
   if (st != AWQ_OK) return st;
@@ -387,6 +387,14 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
   if (st != AWQ_OK) return st;
   const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
   const long long tiles = nst * ((M + BT - 1) / BT);
+  if (KS == 2) {   // CTA pairs: one cluster per tile slot, as many as can be co-resident
+    static ClusterOccCache cache;
+    const int fit = max_active_clusters(kernel, C::kThreads, C::kSmem, 2, dev, cache);
+    if (fit < 1) return AWQ_ERR_UNSUPPORTED;
+    const int clusters = static_cast<int>(std::min<long long>(tiles, fit));
+    return launch_ex(kernel, dim3(2 * clusters, 1, 1), dim3(C::kThreads, 1, 1), dim3(2, 1, 1), C::kSmem, stream,
+                     xmap, qmap, smap, zmap, epi, M, N, K);
+  }
   const int grid = static_cast<int>(std::min<long long>(tiles, static_cast<long long>(CPS) * num_sms));
   return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), dim3(0, 0, 0), C::kSmem, stream, xmap, qmap,
                    smap, zmap, epi, M, N, K);
@@ -407,37 +415,75 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 #define AWQ_GEMM_S64 7
 #endif
 
+// With the K split (KS = 2) the exchange slots (16 KB each) share the shared memory with the ring.
+#ifndef AWQ_GEMM_KS_S256
+#define AWQ_GEMM_KS_S256 3
+#endif
+#ifndef AWQ_GEMM_KS_S128
+#define AWQ_GEMM_KS_S128 5
+#endif
+#ifndef AWQ_GEMM_KS_S64
+#define AWQ_GEMM_KS_S64 6
+#endif
+#ifndef AWQ_GEMM_KS_S32
+#define AWQ_GEMM_KS_S32 8
+#endif
+// Relative cost of a K-split tile beyond half a tile (the partial-sum exchange, the shorter ring).
+#ifndef AWQ_GEMM_KS_OVERHEAD
+#define AWQ_GEMM_KS_OVERHEAD 0.1
+#endif
+
+// Test hook (awq_debug_set_gemm_split): 0 lets the round model choose the K split, 1 or 2 forces it.
+std::atomic<int> g_force_ks{0};
+
 template <int EPI>
 awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  if (M <= 32) return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-  if (M <= 64)
-    return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
-  // Token tile by a round model: the persistent CTAs (one per SM) take tiles round-robin, so a
-  // launch costs ceil(tiles / SMs) rounds, and a tile's time grows only slowly with BT because
-  // dequantizing its 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted
-  // on the Llama-3-8B prefill and Llama-2-70B layers at M = 512 and 2048).
+  // Token tile BT and K split KS by a round model: the persistent CTAs (one per SM; with KS = 2,
+  // one CTA pair per two SMs) take tiles round-robin, so a launch costs ceil(tiles / slots)
+  // rounds, and a tile's time grows only slowly with BT because dequantizing its 128-row weight
+  // block dominates (per-tile time 0.75 + 0.35 BT/256, fitted on the Llama-3-8B prefill and
+  // Llama-2-70B layers at M = 512 and 2048). A K-split tile takes half a tile's time plus the
+  // exchange. BT = 32 serves M <= 32 and BT = 64 M <= 64.
   const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
-  int best_bt = 64;
+  int best_bt = 64, best_ks = 1;
   double best = 1e300;
-  for (int bt : {256, 128, 64}) {
+  const int bts_small[1] = {M <= 32 ? 32 : 64};
+  const int bts_large[3] = {256, 128, 64};
+  const int* bts = M <= 64 ? bts_small : bts_large;
+  const int nbt = M <= 64 ? 1 : 3;
+  const int force = g_force_ks.load();
+  for (int i = 0; i < nbt; ++i) {
+    const int bt = bts[i];
     const long long tiles = nst * ((M + bt - 1) / bt);
-    const double cost = static_cast<double>((tiles + num_sms - 1) / num_sms) * (0.75 + 0.35 * bt / 256.0);
-    if (cost < best - 1e-9) { best = cost; best_bt = bt; }
+    const double t_tile = 0.75 + 0.35 * bt / 256.0;
+    for (int ks = 1; ks <= 2; ++ks) {
+      if (force != 0 && ks != force) continue;
+      const long long slots = std::max(1, num_sms / ks);
+      const double per = ks == 1 ? t_tile : t_tile * (0.5 + AWQ_GEMM_KS_OVERHEAD);
+      const double cost = static_cast<double>((tiles + slots - 1) / slots) * per;
+      if (cost < best - 1e-9) { best = cost; best_bt = bt; best_ks = ks; }
+    }
   }
 #ifdef AWQ_GEMM_FORCE_BT
   best_bt = AWQ_GEMM_FORCE_BT;
 #endif
-  switch (best_bt) {
-    case 256:
-      return launch_gemm_cfg<256, AWQ_GEMM_S256, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
-                                                                      stream);
-    case 128:
-      return launch_gemm_cfg<128, AWQ_GEMM_S128, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms,
-                                                                      stream);
-    default:
-      return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream);
+#define AWQ_GEMM_ARGS x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream
+  if (best_ks == 2) {
+    switch (best_bt) {
+      case 256: return launch_gemm_cfg<256, AWQ_GEMM_KS_S256, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+      case 128: return launch_gemm_cfg<128, AWQ_GEMM_KS_S128, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+      case 64: return launch_gemm_cfg<64, AWQ_GEMM_KS_S64, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+      default: return launch_gemm_cfg<32, AWQ_GEMM_KS_S32, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+    }
   }
+  switch (best_bt) {
+    case 256: return launch_gemm_cfg<256, AWQ_GEMM_S256, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
+    case 128: return launch_gemm_cfg<128, AWQ_GEMM_S128, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
+    case 64: return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
+    default: return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
+  }
+#undef AWQ_GEMM_ARGS
 }
 
 awq_status_t launch_gemm(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr, __half* y, int M,
@@ -812,6 +858,12 @@ awq_status_t awq_debug_drop_first_copy(int enable) {
   const int v = enable ? 1 : 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return AWQ_ERR_CUDA;
   return cudaMemcpyToSymbol(g_debug_drop_first_copy, &v, sizeof(v)) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+awq_status_t awq_debug_set_gemm_split(int ks) {
+  if (ks < 0 || ks > 2) return AWQ_ERR_INVALID_ARG;
+  g_force_ks.store(ks);
+  return AWQ_OK;
 }
 
 awq_status_t awq_debug_set_wait_budget_ns(unsigned long long ns) {
