@@ -75,7 +75,7 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(
 // KS: CTAs that share one output tile, each over its part of K (a cluster of KS = 2 CTAs; rank 1
 // pushes its fp32 partial sums into rank 0's shared memory with asynchronous stores that count
 // down rank 0's mbarrier, 32 columns at a time, through an exchange buffer of two or more slots).
-template <int BT, int STAGES, int NDQ, int CPS = 1, int KS = 1>
+template <int BT, int STAGES, int NDQ, int CPS = 1, int KS = 1, int EPI = kEpiPlain>
 struct GemmCfg {
   static_assert(BT % 32 == 0 && BT >= 32 && BT <= 256, "token tile");
   static_assert(CPS == 1 || CPS == 2, "CTAs per SM");
@@ -86,7 +86,8 @@ struct GemmCfg {
   static constexpr int kRawQ = kSuperChunkWords * 4;        // 4096 B
   static constexpr int kRawS = 8 * 16 * 2;                  // 256 B
   static constexpr int kZeroBytes = 8 * 16;                 // 128 B: zeros of the group pair, 8 tiles
-  static constexpr int kRawZ = 256;                         // zeros slot: two 128-byte-aligned halves
+  // zeros slot: kEpiSiluMul loads the gate and the up tiles' zeros into two 128-byte-aligned halves
+  static constexpr int kRawZ = EPI == kEpiSiluMul ? 256 : 128;
   static constexpr int kTx = kB + kRawQ + kRawS + kZeroBytes;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kA;
@@ -120,11 +121,11 @@ struct GemmCfg {
 };
 
 template <int BT, int STAGES, int NDQ, int CPS, int EPI, int KS = 1>
-__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS>::kThreads, CPS)
+__global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThreads, CPS)
     awq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
                     const EpiArgs epi, int M, int N, int K) {
-  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);

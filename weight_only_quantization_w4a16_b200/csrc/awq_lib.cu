@@ -375,7 +375,7 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
 template <int BT, int STAGES, int NDQ, int CPS = 1, int EPI = kEpiPlain, int KS = 1>
 awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS>;
+  using C = GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>;
   auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS, EPI, KS>;
   static std::atomic<uint64_t> smem_done{0};
   awq_status_t st = ensure_smem(kernel, C::kSmem, dev, smem_done);
@@ -417,7 +417,7 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 
 // With the K split (KS = 2) the exchange slots (16 KB each) share the shared memory with the ring.
 #ifndef AWQ_GEMM_KS_S256
-#define AWQ_GEMM_KS_S256 3
+#define AWQ_GEMM_KS_S256 4
 #endif
 #ifndef AWQ_GEMM_KS_S128
 #define AWQ_GEMM_KS_S128 5
@@ -471,7 +471,8 @@ awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* 
 #define AWQ_GEMM_ARGS x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream
   if (best_ks == 2) {
     switch (best_bt) {
-      case 256: return launch_gemm_cfg<256, AWQ_GEMM_KS_S256, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+      case 256:   // kEpiSiluMul's wider zeros slots leave room for 3 stages only
+        return launch_gemm_cfg<256, EPI == kEpiSiluMul ? 3 : AWQ_GEMM_KS_S256, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
       case 128: return launch_gemm_cfg<128, AWQ_GEMM_KS_S128, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
       case 64: return launch_gemm_cfg<64, AWQ_GEMM_KS_S64, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
       default: return launch_gemm_cfg<32, AWQ_GEMM_KS_S32, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
