@@ -552,11 +552,15 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(oracle_decode_inputs(wl, M)) if decode else None
 
+    config = bench_config(wl, M, n_sets, set_bytes / 1e6)
+    if not decode:   # the token tile and K split the prefill kernel took for each layer
+        config["plan"] = [{"layer": l.name, "token_tile": bt, "k_split": ks}
+                          for l in wl.layers for bt, ks in [P.awq_gemm_plan(M, l.N, l.K)]]
     line = {
         "metric": metric_name(M), "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
         "warmup": W_steps, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": bench_config(wl, M, n_sets, set_bytes / 1e6), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": K_steps * len(L),
         "clocks": clocks.summary(t_wall0, t_wall1),
         "repeats": {"ms_per_step": [m / K_steps for m in rep_ms], "median_ms_per_step": statistics.median(rep_ms) / K_steps,

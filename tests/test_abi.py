@@ -89,6 +89,50 @@ def test_gemm_split_hook_is_host_only(lib):
         assert lib.awq_debug_set_gemm_split(ok) == 0
 
 
+# The prefill kernel's launch plan on 148 SMs for the Llama-3-8B prefill layers: each entry is
+# the fastest form, or within 5% of it, in a per-layer sweep that forced every token tile with
+# the K split off and on (CUDA events, B200).
+PLAN_CASES = [
+    # (M, N, K, token tile, K split)
+    (512, 6144, 4096, 256, 1),    # q/k/v: 96 tiles, a split would add a round
+    (512, 4096, 4096, 256, 2),    # o_proj: 64 tiles
+    (512, 28672, 4096, 256, 1),   # gate/up: 448 tiles
+    (512, 4096, 14336, 256, 2),   # down_proj: 64 tiles
+    (128, 6144, 4096, 128, 2),
+    (128, 4096, 4096, 64, 2),
+    (128, 28672, 4096, 128, 1),
+    (128, 4096, 14336, 64, 2),
+    (2048, 28672, 4096, 256, 1),
+    (32, 4096, 4096, 32, 2),
+]
+
+
+@pytest.mark.parametrize("M,N,K,bt,ks", PLAN_CASES)
+def test_gemm_plan_matches_measured_choices(lib, M, N, K, bt, ks):
+    import weight_only_quantization_w4a16_b200 as P
+    assert P.awq_gemm_plan(M, N, K, 0, num_sms=148) == (bt, ks)
+
+
+def test_gemm_plan_hook_and_argument_checks(lib):
+    import weight_only_quantization_w4a16_b200 as P
+    try:
+        P.awq_debug_set_gemm_split(1)
+        assert P.awq_gemm_plan(512, 4096, 14336, 0, num_sms=148)[1] == 1
+        P.awq_debug_set_gemm_split(2)
+        assert P.awq_gemm_plan(2048, 28672, 4096, 0, num_sms=148)[1] == 2
+    finally:
+        P.awq_debug_set_gemm_split(0)
+    bt, ks = ctypes.c_int(), ctypes.c_int()
+    ref = (ctypes.byref(bt), ctypes.byref(ks))
+    assert lib.awq_gemm_plan(0, 16, 128, 0, 148, *ref) == 1
+    assert lib.awq_gemm_plan(1, 16, 100, 0, 148, *ref) == 1
+    assert lib.awq_gemm_plan(1, 16, 128, 3, 148, *ref) == 1
+    assert lib.awq_gemm_plan(1, 16, 128, 0, 0, *ref) == 1
+    assert lib.awq_gemm_plan(1, 48, 128, 2, 148, *ref) == 1       # SiLU: N = 2 I, I % 16 == 0
+    assert lib.awq_gemm_plan(1, 16, 128, 0, 148, None, None) == 1
+    assert lib.awq_gemm_plan(64, 64, 128, 2, 148, *ref) == 0 and (bt.value, ks.value) == (64, 2)
+
+
 def test_quantize_variant_argument_checks(lib):
     """awq_quantize rejects unbuilt configurations before any CUDA call (no GPU needed)."""
     V = ctypes.c_void_p

@@ -76,6 +76,7 @@ _SIGS = {
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
     "awq_debug_drop_first_copy": ([_I], _I),
     "awq_debug_set_gemm_split": ([_I], _I),
+    "awq_gemm_plan": ([_I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
 }
 
 
@@ -427,6 +428,18 @@ def awq_debug_set_wait_budget_ns(ns: int) -> None:
 
 def awq_debug_drop_first_copy(enable: bool) -> None:
     _check("awq_debug_drop_first_copy", load_library().awq_debug_drop_first_copy(int(bool(enable))))
+
+
+def awq_gemm_plan(M: int, N: int, K: int, epilogue: int = 0, num_sms: Optional[int] = None) -> Tuple[int, int]:
+    """(token tile, K split) that the prefill kernel takes for this shape (host-only). epilogue: 0
+    plain, 1 q/k/v split, 2 gate/up SiLU*up; num_sms defaults to the current CUDA device's."""
+    if num_sms is None:
+        import torch
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    bt, ks = ctypes.c_int(0), ctypes.c_int(0)
+    _check("awq_gemm_plan", load_library().awq_gemm_plan(int(M), int(N), int(K), int(epilogue), int(num_sms),
+                                                          ctypes.byref(bt), ctypes.byref(ks)))
+    return bt.value, ks.value
 
 
 def awq_debug_set_gemm_split(ks: int) -> None:

@@ -436,23 +436,20 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 // Test hook (awq_debug_set_gemm_split): 0 lets the round model choose the K split, 1 or 2 forces it.
 std::atomic<int> g_force_ks{0};
 
-template <int EPI>
-awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
-                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  // Token tile BT and K split KS by a round model: the persistent CTAs (one per SM; with KS = 2,
-  // one CTA pair per two SMs) take tiles round-robin, so a launch costs ceil(tiles / slots)
-  // rounds, and a tile's time grows only slowly with BT because dequantizing its 128-row weight
-  // block dominates (per-tile time 0.75 + 0.35 BT/256, fitted on the Llama-3-8B prefill and
-  // Llama-2-70B layers at M = 512 and 2048). A K-split tile takes half a tile's time plus the
-  // exchange. BT = 32 serves M <= 32 and BT = 64 M <= 64.
-  const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
+// Token tile BT and K split KS of the prefill kernel by a round model: the persistent CTAs (one
+// per SM; with KS = 2, one CTA pair per two SMs) take tiles round-robin, so a launch costs
+// ceil(tiles / slots) rounds, and a tile's time grows only slowly with BT because dequantizing its
+// 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted on the Llama-3-8B
+// prefill and Llama-2-70B layers at M = 512 and 2048). A K-split tile takes half a tile's time
+// plus the exchange. BT = 32 serves M <= 32 and BT = 64 M <= 64. `force` (0, 1 or 2) fixes KS.
+void gemm_plan(int M, int N, int epi, int num_sms, int force, int* bt_out, int* ks_out) {
+  const long long nst = epi == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
   int best_bt = 64, best_ks = 1;
   double best = 1e300;
   const int bts_small[1] = {M <= 32 ? 32 : 64};
   const int bts_large[3] = {256, 128, 64};
   const int* bts = M <= 64 ? bts_small : bts_large;
   const int nbt = M <= 64 ? 1 : 3;
-  const int force = g_force_ks.load();
   for (int i = 0; i < nbt; ++i) {
     const int bt = bts[i];
     const long long tiles = nst * ((M + bt - 1) / bt);
@@ -465,6 +462,15 @@ awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* 
       if (cost < best - 1e-9) { best = cost; best_bt = bt; best_ks = ks; }
     }
   }
+  *bt_out = best_bt;
+  *ks_out = best_ks;
+}
+
+template <int EPI>
+awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+  int best_bt, best_ks;
+  gemm_plan(M, N, EPI, num_sms, g_force_ks.load(), &best_bt, &best_ks);
 #ifdef AWQ_GEMM_FORCE_BT
   best_bt = AWQ_GEMM_FORCE_BT;
 #endif
@@ -859,6 +865,15 @@ awq_status_t awq_debug_drop_first_copy(int enable) {
   const int v = enable ? 1 : 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return AWQ_ERR_CUDA;
   return cudaMemcpyToSymbol(g_debug_drop_first_copy, &v, sizeof(v)) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+awq_status_t awq_gemm_plan(int M, int N, int K, int epilogue, int num_sms, int* token_tile, int* k_split) {
+  if (!token_tile || !k_split || M < 1 || K < kGroup || K % kGroup != 0 || !rows_ok(N, K) || num_sms < 1 ||
+      epilogue < kEpiPlain || epilogue > kEpiSiluMul)
+    return AWQ_ERR_INVALID_ARG;
+  if (epilogue == kEpiSiluMul && N % 32 != 0) return AWQ_ERR_INVALID_ARG;
+  gemm_plan(M, N, epilogue, num_sms, g_force_ks.load(), token_tile, k_split);
+  return AWQ_OK;
 }
 
 awq_status_t awq_debug_set_gemm_split(int ks) {
