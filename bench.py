@@ -554,8 +554,8 @@ def run_ours(args, world, rank, local):
 
     config = bench_config(wl, M, n_sets, set_bytes / 1e6)
     if not decode:   # the token tile and K split the prefill kernel took for each layer
-        config["plan"] = [{"layer": l.name, "token_tile": bt, "k_split": ks}
-                          for l in wl.layers for bt, ks in [P.awq_gemm_plan(M, l.N, l.K)]]
+        config["plan"] = [{"layer": l.name, "token_tile": bt, "k_split": ks, "split_tiles": nsplit}
+                          for l in wl.layers for bt, ks, nsplit in [P.awq_gemm_plan(M, l.N, l.K)]]
     line = {
         "metric": metric_name(M), "value": value, "unit": unit, "n_gpus": world, "steps": K_steps,
         "warmup": W_steps, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

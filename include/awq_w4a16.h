@@ -312,21 +312,26 @@ AWQ_API awq_status_t awq_debug_drop_first_copy(int enable);
 
 /* The launch plan awq_w4a16_gemm (and the fused prefill entry points)
  * would take for an M x K by K x N layer on a GPU with num_sms SMs: the
- * token tile (*token_tile: 32, 64, 128 or 256 tokens per tile) and the K
- * split (*k_split: 1, or 2 when the two CTAs of a cluster share each
- * tile, each over half of K). epilogue: 0 plain, 1 q/k/v split, 2 gate/up
- * SiLU·up (N = 2 I, I a multiple of 16). Host-only; honours
- * awq_debug_set_gemm_split. AWQ_ERR_INVALID_ARG for null outputs or the
- * shapes the linear entry points reject. */
-AWQ_API awq_status_t awq_gemm_plan(int M, int N, int K, int epilogue, int num_sms, int* token_tile, int* k_split);
+ * token tile (*token_tile: 32, 64, 128 or 256 tokens per tile), the K
+ * split (*k_split: 1, or 2 when the two CTAs of a thread-block cluster
+ * share tiles, each over half of K) and *split_tiles, how many of the
+ * layer's tiles are shared that way (all of them, or only those left
+ * for the last round after whole rounds of one tile per SM). epilogue:
+ * 0 plain, 1 q/k/v split, 2 gate/up SiLU·up (N = 2 I, I a multiple of
+ * 16). Host-only; honours awq_debug_set_gemm_split. AWQ_ERR_INVALID_ARG
+ * for null outputs or the shapes the linear entry points reject. */
+AWQ_API awq_status_t awq_gemm_plan(int M, int N, int K, int epilogue, int num_sms, int* token_tile, int* k_split,
+                                   long long* split_tiles);
 
 /* Test hook: the prefill kernel's K split. 0 (the default) lets the
  * library's round model choose, per launch, whether the two CTAs of a
- * thread-block cluster share each output tile (each over half of K, their
- * fp32 partial sums added in a fixed order); 1 never splits, 2 always
- * splits. Results agree within fp32 rounding of the split sum. Host-side
- * setting for all devices, read at each launch; AWQ_ERR_INVALID_ARG for
- * other values. */
+ * thread-block cluster share output tiles (each over half of K, their
+ * fp32 partial sums added in a fixed order); 1 never splits, 2 splits
+ * every tile, 3 takes the mixed form (whole rounds of one tile per CTA,
+ * then the remaining tiles split) on a grid of 3 CTA pairs, so that small
+ * layers run both kinds of work item. Results agree within fp32 rounding
+ * of the split sum. Host-side setting for all devices, read at each
+ * launch; AWQ_ERR_INVALID_ARG for other values. */
 AWQ_API awq_status_t awq_debug_set_gemm_split(int ks);
 
 #ifdef __cplusplus

@@ -83,54 +83,62 @@ def test_check_config_against_page_configs(lib):
 
 def test_gemm_split_hook_is_host_only(lib):
     """The K-split test hook takes 0, 1 or 2 and touches no device."""
-    for bad in (-1, 3, 100):
+    for bad in (-1, 4, 100):
         assert lib.awq_debug_set_gemm_split(bad) == 1
-    for ok in (2, 1, 0):
+    for ok in (3, 2, 1, 0):
         assert lib.awq_debug_set_gemm_split(ok) == 0
 
 
 # The prefill kernel's launch plan on 148 SMs for the Llama-3-8B prefill layers: each entry is
-# the fastest form, or within 5% of it, in a per-layer sweep that forced every token tile with
-# the K split off and on (CUDA events, B200).
+# the fastest form, or within 5% of it, in per-layer sweeps that forced every token tile with the
+# K split off, on for every tile, and on for the last round's tiles only (CUDA events, B200).
 PLAN_CASES = [
-    # (M, N, K, token tile, K split)
-    (512, 6144, 4096, 256, 1),    # q/k/v: 96 tiles, a split would add a round
-    (512, 4096, 4096, 256, 2),    # o_proj: 64 tiles
-    (512, 28672, 4096, 256, 1),   # gate/up: 448 tiles
-    (512, 4096, 14336, 256, 2),   # down_proj: 64 tiles
-    (128, 6144, 4096, 128, 2),
-    (128, 4096, 4096, 64, 2),
-    (128, 28672, 4096, 128, 1),
-    (128, 4096, 14336, 64, 2),
-    (2048, 28672, 4096, 256, 1),
-    (32, 4096, 4096, 32, 2),
+    # (M, N, K, token tile, K split, split tiles)
+    (512, 6144, 4096, 256, 1, 0),       # q/k/v: 96 tiles, a split would add a round
+    (512, 4096, 4096, 256, 2, 64),      # o_proj: 64 tiles, all split
+    (512, 28672, 4096, 256, 2, 4),      # gate/up: 3 whole rounds of 148 tiles, the last 4 split
+    (512, 4096, 14336, 256, 2, 64),     # down_proj: 64 tiles, all split
+    (128, 6144, 4096, 128, 2, 48),
+    (128, 4096, 4096, 64, 2, 64),
+    (128, 28672, 4096, 128, 1, 0),
+    (128, 4096, 14336, 64, 2, 64),
+    (2048, 28672, 4096, 256, 1, 0),     # 12.1 rounds: splitting the last 16 tiles measured no gain
+    (2048, 6144, 4096, 256, 1, 0),      # 384 tiles: 88 left over, more than 74 pairs
+    (32, 4096, 4096, 32, 2, 32),
+    (512, 28672, 8192, 256, 2, 4),      # Llama-2-70B gate/up: 234.5 us against 256.7 without the split
+    (512, 8192, 28672, 256, 1, 0),      # Llama-2-70B down: 128 tiles, one round
 ]
 
 
-@pytest.mark.parametrize("M,N,K,bt,ks", PLAN_CASES)
-def test_gemm_plan_matches_measured_choices(lib, M, N, K, bt, ks):
+@pytest.mark.parametrize("M,N,K,bt,ks,nsplit", PLAN_CASES)
+def test_gemm_plan_matches_measured_choices(lib, M, N, K, bt, ks, nsplit):
     import weight_only_quantization_w4a16_b200 as P
-    assert P.awq_gemm_plan(M, N, K, 0, num_sms=148) == (bt, ks)
+    assert P.awq_gemm_plan(M, N, K, 0, num_sms=148) == (bt, ks, nsplit)
 
 
 def test_gemm_plan_hook_and_argument_checks(lib):
     import weight_only_quantization_w4a16_b200 as P
     try:
         P.awq_debug_set_gemm_split(1)
-        assert P.awq_gemm_plan(512, 4096, 14336, 0, num_sms=148)[1] == 1
+        assert P.awq_gemm_plan(512, 4096, 14336, 0, num_sms=148)[1:] == (1, 0)
         P.awq_debug_set_gemm_split(2)
-        assert P.awq_gemm_plan(2048, 28672, 4096, 0, num_sms=148)[1] == 2
+        assert P.awq_gemm_plan(2048, 28672, 4096, 0, num_sms=148)[1:] == (2, 224 * 8)
+        # form 3 (3 CTA pairs): the GPU tests' shape 300 x 1000 x 1280 takes whole-tile rounds and
+        # split tiles in one launch
+        P.awq_debug_set_gemm_split(3)
+        bt, ks, nsplit = P.awq_gemm_plan(300, 1000, 1280, 0, num_sms=148)
+        assert ks == 2 and 0 < nsplit < 8 * -(-300 // bt)
     finally:
         P.awq_debug_set_gemm_split(0)
-    bt, ks = ctypes.c_int(), ctypes.c_int()
-    ref = (ctypes.byref(bt), ctypes.byref(ks))
+    bt, ks, ns = ctypes.c_int(), ctypes.c_int(), ctypes.c_longlong()
+    ref = (ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(ns))
     assert lib.awq_gemm_plan(0, 16, 128, 0, 148, *ref) == 1
     assert lib.awq_gemm_plan(1, 16, 100, 0, 148, *ref) == 1
     assert lib.awq_gemm_plan(1, 16, 128, 3, 148, *ref) == 1
     assert lib.awq_gemm_plan(1, 16, 128, 0, 0, *ref) == 1
     assert lib.awq_gemm_plan(1, 48, 128, 2, 148, *ref) == 1       # SiLU: N = 2 I, I % 16 == 0
-    assert lib.awq_gemm_plan(1, 16, 128, 0, 148, None, None) == 1
-    assert lib.awq_gemm_plan(64, 64, 128, 2, 148, *ref) == 0 and (bt.value, ks.value) == (64, 2)
+    assert lib.awq_gemm_plan(1, 16, 128, 0, 148, None, None, None) == 1
+    assert lib.awq_gemm_plan(64, 64, 128, 2, 148, *ref) == 0 and (bt.value, ks.value, ns.value) == (64, 2, 1)
 
 
 def test_quantize_variant_argument_checks(lib):

@@ -1,9 +1,11 @@
 """GPU parity of the prefill kernel's K split (a CTA pair per output tile, each over half of K,
 rank 1's fp32 partial sums pushed into rank 0's shared memory) against the oracle.
 
-awq_debug_set_gemm_split forces the split off (1) or on (2) so that both forms run on the same
-shapes, token tiles 32 to 256, every epilogue, and K from one group pair upward; the split form
-must be deterministic and within the same bars as the unsplit one.
+awq_debug_set_gemm_split forces the split off (1), on for every tile (2), or the mixed form (3:
+whole rounds of one tile per CTA, then the remaining tiles split, on a grid of 3 CTA pairs so
+that small layers take both kinds of work item). Every form runs on the same shapes, token tiles
+32 to 256, every epilogue, and K from one group pair upward; the split forms must be
+deterministic and within the same bars as the unsplit one.
 """
 import numpy as np
 import pytest
@@ -39,29 +41,31 @@ def _prep(x, W):
 # M picks the token tile (32, 64, then the round model's 64/128/256); K = 128 gives each CTA of
 # the pair a single 64-k step.
 @pytest.mark.parametrize("M", [5, 33, 100, 300, 513])
-@pytest.mark.parametrize("N,K", [(256, 128), (200, 384), (1000, 1280), (136, 2304)])
+@pytest.mark.parametrize("N,K", [(256, 128), (200, 384), (1000, 1280), (136, 2304), (896, 640)])
 def test_split_matches_oracle_and_unsplit(split, M, N, K):
     P = lib()
     x, W = workloads.random_case(211 + M, M, N, K)
     r = O.reference_forward(x, W)
     xs, pk = _prep(x, W)
     out = {}
-    for ks in (1, 2):
+    for ks in (1, 2, 3):
         split(ks)
         y = host(P.awq_w4a16_gemm(xs, *pk, N))
         assert P.awq_poll_device_status() == P.AWQ_OK
         assert_tolerance(y.astype(np.float64), r["y"], f"gemm ks={ks} M={M} N={N} K={K}")
         assert_tight(y, r["y"], rel=2.0 ** -10, abs_rms=3e-3, what=f"gemm ks={ks}")
         out[ks] = y
-    split(2)
-    again = host(P.awq_w4a16_gemm(xs, *pk, N))
-    assert np.array_equal(f16_bits(again), f16_bits(out[2])), "split form not deterministic"
+    for ks in (2, 3):
+        split(ks)
+        again = host(P.awq_w4a16_gemm(xs, *pk, N))
+        assert np.array_equal(f16_bits(again), f16_bits(out[ks])), f"split form {ks} not deterministic"
 
 
+@pytest.mark.parametrize("ks", [2, 3])
 @pytest.mark.parametrize("M", [40, 300])
-def test_split_fused_epilogues(split, M):
+def test_split_fused_epilogues(split, M, ks):
     P = lib()
-    split(2)
+    split(ks)
     Nq, Nkv, K = 512, 128, 1280
     x, W = workloads.random_case(231 + M, M, Nq + 2 * Nkv, K)
     r = O.reference_forward(x, W)
@@ -100,5 +104,5 @@ def test_split_full_size_down_proj_sampled(split):
 
 def test_split_hook_rejects_bad_values():
     P = lib()
-    for bad in (-1, 3):
+    for bad in (-1, 4):
         assert P.load_library().awq_debug_set_gemm_split(bad) == P.AWQ_ERR_INVALID_ARG

@@ -76,7 +76,8 @@ _SIGS = {
     "awq_debug_set_wait_budget_ns": ([ctypes.c_ulonglong], _I),
     "awq_debug_drop_first_copy": ([_I], _I),
     "awq_debug_set_gemm_split": ([_I], _I),
-    "awq_gemm_plan": ([_I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "awq_gemm_plan": ([_I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_longlong)],
+                      _I),
 }
 
 
@@ -430,20 +431,21 @@ def awq_debug_drop_first_copy(enable: bool) -> None:
     _check("awq_debug_drop_first_copy", load_library().awq_debug_drop_first_copy(int(bool(enable))))
 
 
-def awq_gemm_plan(M: int, N: int, K: int, epilogue: int = 0, num_sms: Optional[int] = None) -> Tuple[int, int]:
-    """(token tile, K split) that the prefill kernel takes for this shape (host-only). epilogue: 0
-    plain, 1 q/k/v split, 2 gate/up SiLU*up; num_sms defaults to the current CUDA device's."""
+def awq_gemm_plan(M: int, N: int, K: int, epilogue: int = 0, num_sms: Optional[int] = None) -> Tuple[int, int, int]:
+    """(token tile, K split, split tiles) that the prefill kernel takes for this shape (host-only).
+    epilogue: 0 plain, 1 q/k/v split, 2 gate/up SiLU*up; num_sms defaults to the current device's."""
     if num_sms is None:
         import torch
         num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    bt, ks = ctypes.c_int(0), ctypes.c_int(0)
+    bt, ks, nsplit = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_longlong(0)
     _check("awq_gemm_plan", load_library().awq_gemm_plan(int(M), int(N), int(K), int(epilogue), int(num_sms),
-                                                          ctypes.byref(bt), ctypes.byref(ks)))
-    return bt.value, ks.value
+                                                          ctypes.byref(bt), ctypes.byref(ks), ctypes.byref(nsplit)))
+    return bt.value, ks.value, nsplit.value
 
 
 def awq_debug_set_gemm_split(ks: int) -> None:
-    """Prefill K split: 0 chooses per launch, 1 never splits, 2 always splits (a CTA pair per tile)."""
+    """Prefill K split: 0 chooses per launch, 1 never splits, 2 splits every tile across a CTA pair,
+    3 the mixed form (whole rounds, then the rest split) on a grid of 3 CTA pairs (a test form)."""
     _check("awq_debug_set_gemm_split", load_library().awq_debug_set_gemm_split(int(ks)))
 
 

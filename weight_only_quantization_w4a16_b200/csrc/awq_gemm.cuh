@@ -120,11 +120,20 @@ struct GemmCfg {
   static_assert(CPS == 1 || (kSmem + 1024) * 2 <= 233472, "two CTAs per SM must fit in shared memory");
 };
 
+// One work item of a CTA: a tile over 64-k steps [kb0, kb1), shared with the other CTA of the
+// cluster when `split`.
+struct GemmWork {
+  int tile, kb0, kb1;
+  bool split;
+};
+
+// solo (KS = 2 only): rounds in which every CTA of the grid takes a tile of its own over all of K
+// before the remaining tiles are split across the CTA pairs (0: every tile is split).
 template <int BT, int STAGES, int NDQ, int CPS, int EPI, int KS = 1>
 __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThreads, CPS)
     awq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_s, const __grid_constant__ CUtensorMap tmap_z,
-                    const EpiArgs epi, int M, int N, int K) {
+                    const EpiArgs epi, int M, int N, int K, int solo) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -148,10 +157,27 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
   const int MTT = (M + BT - 1) / BT;
   const int ntiles = NST * MTT;
   const int KB = K / kKTile;
-  // KS = 2: the CTA pair of a cluster takes the same tiles, rank r the 64-k steps [kb0, kb1)
+  // The CTA's work items in order; every role walks the same sequence. KS = 1: tiles blockIdx.x,
+  // + gridDim.x, ... over all of K. KS = 2: first `solo` rounds of one tile per CTA over all of K,
+  // then the remaining tiles striped over the clusters, the CTA pair of a cluster sharing each
+  // (rank r: steps [r KB / 2, (r + 1) KB / 2)).
+  const int G = static_cast<int>(gridDim.x);
   const int rank = KS == 2 ? static_cast<int>(blockIdx.x % KS) : 0;
-  const int tile0 = static_cast<int>(blockIdx.x) / KS, tstep = static_cast<int>(gridDim.x) / KS;
-  const int kb0 = rank * KB / KS, kb1 = (rank + 1) * KB / KS;
+  const int nsolo = KS == 2 ? solo : 0;
+  auto work = [&](int i, GemmWork& w) -> bool {
+    if (KS == 1 || i < nsolo) {
+      w.tile = KS == 1 ? static_cast<int>(blockIdx.x) + i * G : i * G + static_cast<int>(blockIdx.x);
+      w.kb0 = 0;
+      w.kb1 = KB;
+      w.split = false;
+    } else {
+      w.tile = nsolo * G + static_cast<int>(blockIdx.x) / KS + (i - nsolo) * (G / KS);
+      w.kb0 = rank * KB / KS;
+      w.kb1 = (rank + 1) * KB / KS;
+      w.split = true;
+    }
+    return w.tile < ntiles;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -200,9 +226,10 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_par = 0;   // per stage: loaded at least once / parity of last load
       bool ok = true;
-      for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
-        const int st = tile % NST, mt = tile / NST;
-        for (int kb = kb0; kb < kb1; ++kb) {
+      GemmWork w;
+      for (int i = 0; ok && work(i, w); ++i) {
+        const int st = w.tile % NST, mt = w.tile / NST;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, s_abort, budget)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::kTx);
           if (EPI == kEpiSiluMul) {   // 4-tile boxes: gate tiles to slots 0..3, up tiles to slots 4..7
@@ -239,13 +266,14 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
       uint32_t phase = 0;
       bool ok = true, any = false;
       int it = 0;
-      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
+      GemmWork w;
+      for (; ok && work(it, w); ++it) {
         const int b = it % C::kNAcc;
         const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
         if (!mbar_wait_bounded(&accempty[b], (use & 1) ^ 1, s_abort, budget)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * BT);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, s_abort, budget) ||
               !mbar_wait_bounded(&aready[stage], phase, s_abort, budget)) { ok = false; break; }
           tc_fence_after();
@@ -254,7 +282,7 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
 #pragma unroll
           for (int kk = 0; kk < kKTile / 16; ++kk)
             tc_mma_f16(d_tmem, smem_desc_sw128(a0 + 32 * kk), smem_desc_sw128(b0 + 32 * kk), idesc,
-                       (kb != kb0 || kk != 0) ? 1u : 0u);
+                       (kb != w.kb0 || kk != 0) ? 1u : 0u);
           any = true;
           tc_commit(&empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -273,8 +301,9 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
-      for (int kb = kb0; kb < kb1; ++kb) {
+    GemmWork w;
+    for (int i = 0; ok && work(i, w); ++i) {
+      for (int kb = w.kb0; kb < w.kb1; ++kb) {
         // warp-uniform result: the code below needs the whole warp
         if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&full[stage], phase, s_abort, budget))) { ok = false; break; }
         const uint32_t* rq = reinterpret_cast<const uint32_t*>(smem + C::kOffQ + stage * C::kRawQ);
@@ -323,8 +352,9 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
     bool ok = true;
     int it = 0;
     uint32_t xq = 0;   // KS = 2: exchange chunks so far (slot xq % X, phase parity (xq / X) & 1)
-    for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
-      const int st = tile % NST, mt = tile / NST;
+    GemmWork w;
+    for (; ok && work(it, w); ++it) {
+      const int st = w.tile % NST, mt = w.tile / NST;
       const int b = it % C::kNAcc;
       const uint32_t use = static_cast<uint32_t>(it / C::kNAcc);
       if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&accfull[b], use & 1, s_abort, budget))) { ok = false; break; }
@@ -338,11 +368,12 @@ __global__ void __launch_bounds__(GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>::kThrea
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(32 * e) << 16) + static_cast<uint32_t>(b * BT + 32 * cc), v);
         tc_wait_ld();
-        if constexpr (KS == 2) {
+        if (KS == 2 && w.split) {
           // row 32 e + lane of the chunk: 8 16-byte pieces, piece j at position j ^ (lane & 7) of
           // the row's 128 bytes (the 8 lanes of a shared-memory phase hit distinct banks)
-          const int xs = static_cast<int>(xq % C::kXSlots);
-          const uint32_t xpar = (xq / C::kXSlots) & 1;
+          constexpr int kXS = C::kXSlots > 0 ? C::kXSlots : 1;
+          const int xs = static_cast<int>(xq % kXS);
+          const uint32_t xpar = (xq / kXS) & 1;
           ++xq;
           uint8_t* xrow = smem + C::kOffX + xs * C::kXChunk + (32 * e + lane) * 128;
           if (rank == 1) {

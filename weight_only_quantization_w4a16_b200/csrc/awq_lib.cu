@@ -372,9 +372,12 @@ awq_status_t launch_gemv(const __half* x, const uint32_t* qw, const __half* sc, 
 }
 
 // --------------------------------------------------------------------------- prefill dispatch
+// KS = 2: `mixed` runs whole rounds of one tile per CTA first and splits only the tiles left for
+// the last round; `max_clusters` (> 0) caps the grid (a test hook).
 template <int BT, int STAGES, int NDQ, int CPS = 1, int EPI = kEpiPlain, int KS = 1>
 awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
-                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
+                             const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream,
+                             bool mixed = false, int max_clusters = 0) {
   using C = GemmCfg<BT, STAGES, NDQ, CPS, KS, EPI>;
   auto kernel = awq_gemm_kernel<BT, STAGES, NDQ, CPS, EPI, KS>;
   static std::atomic<uint64_t> smem_done{0};
@@ -387,17 +390,21 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
   if (st != AWQ_OK) return st;
   const long long nst = EPI == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
   const long long tiles = nst * ((M + BT - 1) / BT);
-  if (KS == 2) {   // CTA pairs: one cluster per tile slot, as many as can be co-resident
+  if (KS == 2) {   // CTA pairs, as many as can be co-resident
     static ClusterOccCache cache;
-    const int fit = max_active_clusters(kernel, C::kThreads, C::kSmem, 2, dev, cache);
+    int fit = max_active_clusters(kernel, C::kThreads, C::kSmem, 2, dev, cache);
+    if (max_clusters > 0) fit = std::min(fit, max_clusters);
     if (fit < 1) return AWQ_ERR_UNSUPPORTED;
-    const int clusters = static_cast<int>(std::min<long long>(tiles, fit));
+    // mixed: every CTA takes whole tiles for tiles / (2 fit) rounds, the rest are split
+    const int solo = mixed ? static_cast<int>(tiles / (2ll * fit)) : 0;
+    const long long split_tiles = tiles - 2ll * fit * solo;
+    const int clusters = solo > 0 ? fit : static_cast<int>(std::min<long long>(split_tiles, fit));
     return launch_ex(kernel, dim3(2 * clusters, 1, 1), dim3(C::kThreads, 1, 1), dim3(2, 1, 1), C::kSmem, stream,
-                     xmap, qmap, smap, zmap, epi, M, N, K);
+                     xmap, qmap, smap, zmap, epi, M, N, K, solo);
   }
   const int grid = static_cast<int>(std::min<long long>(tiles, static_cast<long long>(CPS) * num_sms));
   return launch_ex(kernel, dim3(grid, 1, 1), dim3(C::kThreads, 1, 1), dim3(0, 0, 0), C::kSmem, stream, xmap, qmap,
-                   smap, zmap, epi, M, N, K);
+                   smap, zmap, epi, M, N, K, 0);
 }
 
 // Compile-time tuning of the prefill kernel: dequantization warps, ring stages per token tile
@@ -432,56 +439,83 @@ awq_status_t launch_gemm_cfg(const __half* x, const uint32_t* qw, const __half* 
 #ifndef AWQ_GEMM_KS_OVERHEAD
 #define AWQ_GEMM_KS_OVERHEAD 0.1
 #endif
+// A split form is taken only when the model prices it at least this factor below the best form
+// without the split: gains smaller than the per-layer sweeps' run-to-run spread (a few percent)
+// did not show up in them (Llama-3-8B gate/up at M = 2048: 3% predicted, 3% lost).
+#ifndef AWQ_GEMM_KS_MARGIN
+#define AWQ_GEMM_KS_MARGIN 1.05
+#endif
 
 // Test hook (awq_debug_set_gemm_split): 0 lets the round model choose the K split, 1 or 2 forces it.
 std::atomic<int> g_force_ks{0};
 
-// Token tile BT and K split KS of the prefill kernel by a round model: the persistent CTAs (one
-// per SM; with KS = 2, one CTA pair per two SMs) take tiles round-robin, so a launch costs
+// Token tile BT and K split of the prefill kernel by a round model: the persistent CTAs (one per
+// SM; with the split, one CTA pair per two SMs) take tiles round-robin, so a launch costs
 // ceil(tiles / slots) rounds, and a tile's time grows only slowly with BT because dequantizing its
 // 128-row weight block dominates (per-tile time 0.75 + 0.35 BT/256, fitted on the Llama-3-8B
-// prefill and Llama-2-70B layers at M = 512 and 2048). A K-split tile takes half a tile's time
-// plus the exchange. BT = 32 serves M <= 32 and BT = 64 M <= 64. `force` (0, 1 or 2) fixes KS.
-void gemm_plan(int M, int N, int epi, int num_sms, int force, int* bt_out, int* ks_out) {
+// prefill and Llama-2-70B layers at M = 512 and 2048). A split tile takes half a tile's time plus
+// the exchange. Three forms: no split; every tile split (ks 2); whole rounds of one tile per SM
+// and only the last round's tiles split (ks 2, mixed). BT = 32 serves M <= 32 and BT = 64 M <= 64.
+// `force`: 0 the model, 1 no split, 2 every tile split, 3 the mixed form on a grid of 3 CTA pairs
+// (a test hook that makes small layers take both kinds of work item).
+struct GemmPlan {
+  int bt, ks;
+  bool mixed;
+  int max_clusters;          // > 0: grid cap (force 3)
+  long long split_tiles;     // tiles split across a CTA pair, on num_sms SMs
+};
+GemmPlan gemm_plan(int M, int N, int epi, int num_sms, int force) {
   const long long nst = epi == kEpiSiluMul ? ceil_div(N / 32, 4) : padded_rows(N) / kSuperRows;
-  int best_bt = 64, best_ks = 1;
+  GemmPlan best_plan = {64, 1, false, 0, 0};
   double best = 1e300;
   const int bts_small[1] = {M <= 32 ? 32 : 64};
   const int bts_large[3] = {256, 128, 64};
   const int* bts = M <= 64 ? bts_small : bts_large;
   const int nbt = M <= 64 ? 1 : 3;
+  const long long pairs = force == 3 ? 3 : std::max(1, num_sms / 2);
+  const long long slots1 = std::max(1, num_sms);
+  auto consider = [&](double cost, const GemmPlan& p) {
+    if (cost < best - 1e-9) { best = cost; best_plan = p; }
+  };
   for (int i = 0; i < nbt; ++i) {
     const int bt = bts[i];
     const long long tiles = nst * ((M + bt - 1) / bt);
-    const double t_tile = 0.75 + 0.35 * bt / 256.0;
-    for (int ks = 1; ks <= 2; ++ks) {
-      if (force != 0 && ks != force) continue;
-      const long long slots = std::max(1, num_sms / ks);
-      const double per = ks == 1 ? t_tile : t_tile * (0.5 + AWQ_GEMM_KS_OVERHEAD);
-      const double cost = static_cast<double>((tiles + slots - 1) / slots) * per;
-      if (cost < best - 1e-9) { best = cost; best_bt = bt; best_ks = ks; }
+    const double t_tile = 0.75 + 0.35 * bt / 256.0, t_split = t_tile * (0.5 + AWQ_GEMM_KS_OVERHEAD);
+    if (force == 0 || force == 1)
+      consider(static_cast<double>((tiles + slots1 - 1) / slots1) * t_tile, {bt, 1, false, 0, 0});
+    const double margin = force == 0 ? AWQ_GEMM_KS_MARGIN : 1.0;
+    if (force == 0 || force == 2)
+      consider(margin * static_cast<double>((tiles + pairs - 1) / pairs) * t_split, {bt, 2, false, 0, tiles});
+    if (force == 0 || force == 3) {
+      const long long solo = tiles / (2 * pairs), rest = tiles - 2 * pairs * solo;
+      if (force == 3 || (solo > 0 && rest > 0))
+        consider(margin * (static_cast<double>(solo) * t_tile +
+                           static_cast<double>((rest + pairs - 1) / pairs) * t_split),
+                 {bt, 2, true, force == 3 ? 3 : 0, rest});
     }
   }
-  *bt_out = best_bt;
-  *ks_out = best_ks;
+  return best_plan;
 }
 
 template <int EPI>
 awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* sc, const uint8_t* zr,
                              const EpiArgs& epi, int M, int N, int K, int dev, int num_sms, cudaStream_t stream) {
-  int best_bt, best_ks;
-  gemm_plan(M, N, EPI, num_sms, g_force_ks.load(), &best_bt, &best_ks);
+  const GemmPlan plan = gemm_plan(M, N, EPI, num_sms, g_force_ks.load());
+  int best_bt = plan.bt;
+  const int best_ks = plan.ks;
 #ifdef AWQ_GEMM_FORCE_BT
   best_bt = AWQ_GEMM_FORCE_BT;
 #endif
 #define AWQ_GEMM_ARGS x, qw, sc, zr, epi, M, N, K, dev, num_sms, stream
+#define AWQ_GEMM_SPLIT_ARGS AWQ_GEMM_ARGS, plan.mixed, plan.max_clusters
   if (best_ks == 2) {
     switch (best_bt) {
       case 256:   // kEpiSiluMul's wider zeros slots leave room for 3 stages only
-        return launch_gemm_cfg<256, EPI == kEpiSiluMul ? 3 : AWQ_GEMM_KS_S256, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
-      case 128: return launch_gemm_cfg<128, AWQ_GEMM_KS_S128, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
-      case 64: return launch_gemm_cfg<64, AWQ_GEMM_KS_S64, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
-      default: return launch_gemm_cfg<32, AWQ_GEMM_KS_S32, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_ARGS);
+        return launch_gemm_cfg<256, EPI == kEpiSiluMul ? 3 : AWQ_GEMM_KS_S256, AWQ_GEMM_NDQ, 1, EPI, 2>(
+            AWQ_GEMM_SPLIT_ARGS);
+      case 128: return launch_gemm_cfg<128, AWQ_GEMM_KS_S128, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_SPLIT_ARGS);
+      case 64: return launch_gemm_cfg<64, AWQ_GEMM_KS_S64, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_SPLIT_ARGS);
+      default: return launch_gemm_cfg<32, AWQ_GEMM_KS_S32, AWQ_GEMM_NDQ, 1, EPI, 2>(AWQ_GEMM_SPLIT_ARGS);
     }
   }
   switch (best_bt) {
@@ -490,6 +524,7 @@ awq_status_t launch_gemm_epi(const __half* x, const uint32_t* qw, const __half* 
     case 64: return launch_gemm_cfg<64, AWQ_GEMM_S64, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
     default: return launch_gemm_cfg<32, 8, AWQ_GEMM_NDQ, 1, EPI>(AWQ_GEMM_ARGS);
   }
+#undef AWQ_GEMM_SPLIT_ARGS
 #undef AWQ_GEMM_ARGS
 }
 
@@ -867,17 +902,21 @@ awq_status_t awq_debug_drop_first_copy(int enable) {
   return cudaMemcpyToSymbol(g_debug_drop_first_copy, &v, sizeof(v)) == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
 }
 
-awq_status_t awq_gemm_plan(int M, int N, int K, int epilogue, int num_sms, int* token_tile, int* k_split) {
-  if (!token_tile || !k_split || M < 1 || K < kGroup || K % kGroup != 0 || !rows_ok(N, K) || num_sms < 1 ||
-      epilogue < kEpiPlain || epilogue > kEpiSiluMul)
+awq_status_t awq_gemm_plan(int M, int N, int K, int epilogue, int num_sms, int* token_tile, int* k_split,
+                           long long* split_tiles) {
+  if (!token_tile || !k_split || !split_tiles || M < 1 || K < kGroup || K % kGroup != 0 || !rows_ok(N, K) ||
+      num_sms < 1 || epilogue < kEpiPlain || epilogue > kEpiSiluMul)
     return AWQ_ERR_INVALID_ARG;
   if (epilogue == kEpiSiluMul && N % 32 != 0) return AWQ_ERR_INVALID_ARG;
-  gemm_plan(M, N, epilogue, num_sms, g_force_ks.load(), token_tile, k_split);
+  const GemmPlan p = gemm_plan(M, N, epilogue, num_sms, g_force_ks.load());
+  *token_tile = p.bt;
+  *k_split = p.ks;
+  *split_tiles = p.split_tiles;
   return AWQ_OK;
 }
 
 awq_status_t awq_debug_set_gemm_split(int ks) {
-  if (ks < 0 || ks > 2) return AWQ_ERR_INVALID_ARG;
+  if (ks < 0 || ks > 3) return AWQ_ERR_INVALID_ARG;
   g_force_ks.store(ks);
   return AWQ_OK;
 }
