@@ -22,7 +22,8 @@
  *                             S = fp16(max(hi-lo, 1e-5)/15), z = clamp(rint(-lo/S), 0, 15),
  *                             q = clamp(rint(w'/S) + z, 0, 15)      (fp32, round half to even)
  *   a3  awq_w4a16_gemv        y[M,N] = x'[M,K] . ((q - z) * S)^T, M <= 32  (fp32 accumulate, fp16 out)
- *   a4  awq_w4a16_gemm        the same for any M (tensor-core prefill kernel)
+ *   a4  awq_w4a16_gemm        the same for any M (tensor-core prefill kernel);
+ *       awq_gemm_plan         its launch plan for a shape (token tile, K split)
  *
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers owned by the caller. The library

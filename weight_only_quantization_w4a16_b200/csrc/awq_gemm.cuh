@@ -22,6 +22,14 @@
 //   warps NDQ..NDQ+3: epilogue — tcgen05.ld of the accumulator (each warp its
 //       32-lane quarter), fp16 convert, coalesced stores of y; two TMEM
 //       accumulators let the epilogue of one tile overlap the next mainloop.
+// K split (KS = 2, clusters of two CTAs): when the tiles are too few to fill
+// the SMs, or a few are left over for a last round, the CTA pair of a cluster
+// shares a tile, rank r running 64-k steps [r KB/2, (r+1) KB/2). Rank 1's
+// epilogue sends its fp32 sums, 32 columns at a time, into rank 0's shared
+// memory with st.async stores that count down an mbarrier of rank 0; rank 0
+// adds them to its own (a fixed order) and stores the tile. A launch may
+// first run whole-tile rounds (one tile per CTA, all of K) and split only the
+// tiles left for the last round: every role walks the same work-item sequence.
 // Every mbarrier wait is bounded by %globaltimer; on expiry the CTA records
 // AWQ_ERR_TIMEOUT in the device status word, every role stops, the producer
 // waits for its copies in flight, the MMA thread for its MMAs, and TMEM is
